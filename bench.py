@@ -1,0 +1,444 @@
+"""Benchmark of the CoSA prefill path (KAP proxy + OSK attention) on B200.
+
+One step = one attention layer's prefill through the whole hot path: the
+proxy (key pooling, query pooling + exact scores + HRM flags + ordered
+selection) and the ordered-skipping attention (page remap in its producer),
+on the 128K-token Llama-3.1-8B-shaped layer (32 query heads, 8 KV heads,
+head_dim 128, pages of 64 tokens in a shuffled pool, stage-1 budget 5%,
+tau = 1e-4).  Inputs are synthetic (seeded), already resident in HBM when
+the timed region starts; the 1.5 GiB of inputs per step exceed the 126 MB L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cosa|reference]
+
+Multi-GPU (torchrun): each rank runs its own layer (independent units, no
+data-path collective); value = total layers / max-over-ranks time.
+The reference arm times the CPU oracle on a bounded sample of the same
+workload and extrapolates to ms per layer.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill sparse-attn ms/layer @128K; effective TFLOP/s; % TC peak; speedup vs dense"
+CONFIG_ID = 3
+BUDGET = 0.05
+TAU = 1e-4
+TAUS = (0.0, 1e-5, 1e-4, 1e-3)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def rank_seed(cfg, rank, world):
+    """Each rank prefills its own independent layer: distinct seeds for N > 1,
+    the workload's own seed at N = 1."""
+    return None if world == 1 else cfg * 1000 + rank
+
+
+def max_over_ranks(value, dist=None, device="cuda"):
+    """Max of a per-rank duration over all ranks (the job's time)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dense_flops(seqlens, Hq, d):
+    return float(sum(4.0 * (L * (L + 1) / 2) * d * Hq for L in seqlens))
+
+
+def workload_config(w):
+    return {"workload": w.name, "seq_len": max(w.seqlens), "batch": w.batch, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "page_size": w.page_size, "pages": "shuffled pool" if w.meta.get("shuffled_pages") else "contiguous",
+            "budget": BUDGET, "tau": TAU,
+            "l2": "inputs larger than L2 (q 1 GiB + k/v pages 512 MiB per step), no flush"}
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU side
+
+def oracle_sample(seq_tokens=16384, seed=CONFIG_ID):
+    """Time the oracle (proxy + OSK) on the first `seq_tokens` tokens of the
+    128K layer shape and extrapolate to a full layer by visited blocks."""
+    from oracle import kap, osk
+    from synth import make_custom
+    from synth.workloads import WORKLOADS
+    spec = dict(WORKLOADS[CONFIG_ID])
+    spec.pop("seqlens")
+    spec.pop("name")
+    w = make_custom([seq_tokens], name="llama8b_128k_prefix", seed=seed, **spec)
+    t0 = time.perf_counter()
+    r = kap.kap_proxy(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, BUDGET)
+    o = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, r["order"],
+                r["count"], TAU)
+    dt = time.perf_counter() - t0
+    b = w.block_size
+    nfull = 131072 // b
+    bp = kap.budget_bp(BUDGET)
+    visited_full = w.num_q_heads * sum(kap.keep_count(n, bp) for n in range(1, nfull + 1))
+    visited_sample = int(o["visited"].sum())
+    ms_layer = dt * 1e3 * visited_full / visited_sample
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return ms_layer, dict(kind="oracle", cores=threads,
+                          sample=f"oracle proxy+OSK on the first {seq_tokens} tokens of the 128K layer shape "
+                                 f"(all 32 heads, budget {BUDGET}, tau {TAU}): {dt:.1f} s for {visited_sample} "
+                                 f"visited blocks, scaled to the layer's {visited_full}")
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    times = []
+    cb = None
+    for _ in range(args.warmup):
+        pass   # the oracle has no warm-up state; warm-up steps are not run to bound the CPU time
+    for _ in range(args.steps):
+        v, cb = oracle_sample(seq_tokens=args.ref_tokens)
+        times.append(v)
+    value = statistics.mean(times)
+    cb["value"] = value
+    cb["unit"] = "ms"
+    line = {"metric": METRIC, "value": value, "unit": "ms", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "llama8b_128k", "seq_len": 131072, "budget": BUDGET, "tau": TAU},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU side
+
+def upload(w, device="cuda"):
+    """Synthetic workload (bf16 bit patterns in numpy) -> device tensors + Batch."""
+    import torch
+    import block_sparse_long_14_b200 as cosa
+
+    def bf16(x):
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(device)
+
+    batch = cosa.Batch(w.seqlens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.page_size,
+                       w.num_pages, w.max_pages_per_seq, device=device)
+    return dict(batch=batch, q=bf16(w.q), k_pages=bf16(w.k_pages), v_pages=bf16(w.v_pages),
+                page_table=torch.from_numpy(np.ascontiguousarray(w.page_table)).to(device))
+
+
+def run_cosa(args, rank, world, local_rank):
+    import torch
+    import block_sparse_long_14_b200 as cosa
+    from synth import make_workload
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    w = make_workload(args.config, seed=rank_seed(args.config, rank, world))
+    d = upload(w)
+    batch = d["batch"]
+    ws, kmax = cosa.alloc_workspace(batch, BUDGET)
+    H, N = w.num_q_heads, batch.total_qblocks
+    sel = dict(order=torch.empty((H, N, kmax), dtype=torch.int32, device="cuda"),
+               count=torch.empty((H, N), dtype=torch.int32, device="cuda"),
+               n_hrm=torch.empty((H, N), dtype=torch.int32, device="cuda"),
+               hrm=torch.empty((H, N, kmax), dtype=torch.uint8, device="cuda"))
+    res = dict(out=torch.empty_like(d["q"]), visited=torch.empty((H, N), dtype=torch.int32, device="cuda"),
+               skipped=torch.empty((H, N), dtype=torch.int32, device="cuda"))
+    stream = torch.cuda.current_stream()
+
+    def step(tau=TAU, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        cosa.proxy(batch, d["q"], d["k_pages"], d["page_table"], BUDGET, kmax, ws, out=sel)
+        if ev is not None:
+            ev[1].record(stream)
+        cosa.attn(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], sel["order"], sel["count"], kmax,
+                  tau, ws, out=res)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    cosa.check(ws)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local_rank) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(ev=evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    cosa.check(ws)
+    elapsed = start.elapsed_time(stop)
+    t_proxy = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    elapsed = max_over_ranks(elapsed, dist)
+    ms_per_step = elapsed / args.steps
+    value = ms_per_step / world          # layers of all ranks run concurrently
+
+    # ---- work accounting (identical every step)
+    visited = int(res["visited"].sum().item())
+    skipped = int(res["skipped"].sum().item())
+    b, dh = w.block_size, w.head_dim
+    tile_flops = 2.0 * b * b * dh
+    exec_flops = tile_flops * (visited + (visited - skipped))
+    pk = peaks()
+    attn_tflops = exec_flops / (t_attn * 1e-3) / 1e12
+    q_bytes = w.q.nbytes
+    k_bytes = w.k_pages.nbytes
+    list_bytes = sum(v.numel() * v.element_size() for v in sel.values())
+    proxy_bytes = q_bytes + k_bytes + list_bytes
+    proxy_gbs = proxy_bytes / (t_proxy * 1e-3) / 1e9
+    dflops = dense_flops(w.seqlens, w.num_q_heads, dh)
+    nqb_rows = sum(((L + b - 1) // b) * (((L + b - 1) // b) + 1) // 2 for L in w.seqlens) * w.num_q_heads
+
+    extra = {}
+    if rank == 0 and world == 1 and not args.quick:
+        # tau sweep (device-timed, same inputs)
+        sweep = {}
+        for tau in TAUS:
+            for _ in range(2):
+                step(tau)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ts = []
+            for _ in range(3):
+                step(tau, ev=e)
+                torch.cuda.synchronize()
+                ts.append((e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])))
+            vis = int(res["visited"].sum().item())
+            sk = int(res["skipped"].sum().item())
+            ta = statistics.mean(x[1] for x in ts)
+            tp = statistics.mean(x[0] for x in ts)
+            sweep[str(tau)] = {"ms": tp + ta, "proxy_ms": tp, "attn_ms": ta, "skip_ratio": sk / vis,
+                               "attn_tflops_executed": tile_flops * (2 * vis - sk) / (ta * 1e-3) / 1e12,
+                               "stage2_budget": (vis - sk) / nqb_rows}
+        extra["tau_sweep"] = sweep
+        cosa.check(ws)
+        # dense reference on the same B200: our OSK at budget 100% / tau 0, and torch SDPA (flash)
+        ws_d, kmax_d = cosa.alloc_workspace(batch, 1.0)
+        sel_d = cosa.proxy(batch, d["q"], d["k_pages"], d["page_table"], 1.0, kmax_d, ws_d)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cosa.attn(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], sel_d["order"], sel_d["count"],
+                  kmax_d, 0.0, ws_d, out=res)
+        e0.record(stream)
+        cosa.attn(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], sel_d["order"], sel_d["count"],
+                  kmax_d, 0.0, ws_d, out=res)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        cosa.check(ws_d)
+        dense_osk_ms = e0.elapsed_time(e1)
+        del sel_d, ws_d
+        sdpa_ms = None
+        try:
+            L = w.seqlens[0]
+            G = w.num_q_heads // w.num_kv_heads
+            qd = d["q"].view(L, w.num_q_heads, dh).transpose(0, 1).unsqueeze(0)
+            kd = torch.randn((1, w.num_kv_heads, L, dh), dtype=torch.bfloat16, device="cuda")
+            vd = torch.randn_like(kd)
+            sdpa = torch.nn.functional.scaled_dot_product_attention
+            sdpa(qd, kd, vd, is_causal=True, enable_gqa=True)
+            e0.record(stream)
+            sdpa(qd, kd, vd, is_causal=True, enable_gqa=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            sdpa_ms = e0.elapsed_time(e1)
+            del kd, vd
+        except Exception as exc:  # library reference only
+            extra["sdpa_error"] = str(exc)[:200]
+        extra["dense"] = {"osk_full_budget_tau0_ms": dense_osk_ms, "torch_sdpa_flash_ms": sdpa_ms,
+                          "dense_tflop": dflops / 1e12}
+        extra["speedup_vs_dense"] = {"vs_osk_dense": dense_osk_ms / ms_per_step,
+                                     "vs_torch_sdpa": (sdpa_ms / ms_per_step) if sdpa_ms else None}
+
+    # ---- end to end through the public API: pinned host inputs in, results out
+    e2e = None
+    if not args.quick:
+        h_q = torch.empty(d["q"].shape, dtype=torch.bfloat16, pin_memory=True)
+        h_k = torch.empty(d["k_pages"].shape, dtype=torch.bfloat16, pin_memory=True)
+        h_v = torch.empty(d["v_pages"].shape, dtype=torch.bfloat16, pin_memory=True)
+        h_t = torch.empty(d["page_table"].shape, dtype=torch.int32, pin_memory=True)
+        h_q.copy_(d["q"])
+        h_k.copy_(d["k_pages"])
+        h_v.copy_(d["v_pages"])
+        h_t.copy_(d["page_table"])
+        h_out = torch.empty(res["out"].shape, dtype=torch.bfloat16, pin_memory=True)
+        h_vis = torch.empty(res["visited"].shape, dtype=torch.int32, pin_memory=True)
+        h_skp = torch.empty_like(h_vis, pin_memory=True)
+
+        def e2e_step():
+            d["q"].copy_(h_q, non_blocking=True)
+            d["k_pages"].copy_(h_k, non_blocking=True)
+            d["v_pages"].copy_(h_v, non_blocking=True)
+            d["page_table"].copy_(h_t, non_blocking=True)
+            step()
+            h_out.copy_(res["out"], non_blocking=True)
+            h_vis.copy_(res["visited"], non_blocking=True)
+            h_skp.copy_(res["skipped"], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        k2 = max(2, min(args.steps, 5))
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(k2):
+            e2e_step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+        el = start.elapsed_time(stop)
+        el = max_over_ranks(el, dist)
+        cosa.check(ws)
+        h2d = h_q.nbytes + h_k.nbytes + h_v.nbytes + h_t.nbytes
+        d2h = h_out.nbytes + h_vis.nbytes + h_skp.nbytes
+        e2e = {"value": el / k2 / world, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": k2}
+
+    if rank != 0:
+        return
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "cosa",
+        "config": {**workload_config(w), "parallelism": f"independent layers x{world}" if world > 1 else "single"},
+        "breakdown_ms": {"proxy": t_proxy, "attn": t_attn},
+        "effective_tflops": dflops / (ms_per_step * 1e-3) / 1e12,
+        "attn_executed_tflops": attn_tflops,
+        "pct_tc_peak": attn_tflops / pk["bf16_sustained"],
+        "proxy_gbs": proxy_gbs,
+        "pct_hbm_proxy": proxy_gbs / pk["hbm_gbs"],
+        "realized_budget": {"stage1": visited / nqb_rows, "stage2": (visited - skipped) / nqb_rows,
+                            "skip_ratio": skipped / visited},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": attn_tflops / pk["bf16_sustained"], "traffic": None,
+                     "kernel": "osk_kernel<128,128>",
+                     "peak_source": f"{pk['source']} bf16_tflops_sustained (kernel timed inside repeated steps)",
+                     "algorithmic": f"{exec_flops:.4e} FLOP per launch = 2*128*128*128 * (visited + kept)"},
+        "proxy_roofline": {"bound": "hbm", "achieved": proxy_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": proxy_gbs / pk["hbm_gbs"], "algorithmic_bytes": proxy_bytes,
+                           "kernels": "kpool + kap_score_select"},
+        "clocks": clocks,
+        "gpu_launches": 3 * args.steps,
+        "e2e": e2e,
+        **extra,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, cb = oracle_sample(seq_tokens=args.ref_tokens)
+        cb["value"] = v
+        cb["unit"] = "ms"
+        line["cpu_baseline"] = cb
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cosa", choices=["cosa", "reference"])
+    ap.add_argument("--config", type=int, default=CONFIG_ID)
+    ap.add_argument("--quick", action="store_true", help="skip the tau sweep, dense reference and e2e legs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=16384)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_cosa(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,306 @@
+// libcosa C ABI: argument checks, workspace layout, TMA tensor maps, launches.
+// The declarations and the contract of each entry point are in include/cosa.h.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "cosa_device.cuh"
+#include "cosa_internal.h"
+
+namespace cosa {
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+constexpr uint32_t kDefaultWaitLimit = 1u << 22;
+std::atomic<uint32_t> g_wait_limit{kDefaultWaitLimit};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int ceil_div(long a, long b) { return static_cast<int>((a + b - 1) / b); }
+
+int budget_bp(float budget) { return static_cast<int>(std::floor(static_cast<double>(budget) * 1e4 + 0.5)); }
+
+int keep_count(long n, int bp) {
+  const long k = (n * bp + 9999) / 10000;
+  return static_cast<int>(k < 1 ? 1 : k);
+}
+
+int next_pow2(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+// Query heads handled together by one proxy CTA: the largest of 4, 2, 1 that divides G.
+int proxy_group(const cosa_shape_t& s) {
+  const int G = s.num_q_heads / s.num_kv_heads;
+  return (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
+}
+
+int check_shape(const cosa_shape_t* s) {
+  if (s == nullptr) return COSA_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->num_q_heads < 1 || s->num_kv_heads < 1 || s->num_pages < 1 || s->total_tokens < 1 ||
+      s->total_qblocks < 1 || s->max_seqlen < 1 || s->max_pages_per_seq < 1)
+    return COSA_ERR_INVALID_ARG;
+  if (s->cu_seqlens == nullptr || s->cu_qblocks == nullptr) return COSA_ERR_INVALID_ARG;
+  if (s->num_q_heads % s->num_kv_heads != 0) return COSA_ERR_INVALID_ARG;
+  if (s->num_q_heads / s->num_kv_heads > 8) return COSA_ERR_UNSUPPORTED;
+  if (s->head_dim != 64 && s->head_dim != 128) return COSA_ERR_UNSUPPORTED;
+  if (s->block_size != 64 && s->block_size != 128) return COSA_ERR_UNSUPPORTED;
+  if (s->page_size < 8 || s->page_size % 8 != 0 || s->block_size % s->page_size != 0) return COSA_ERR_UNSUPPORTED;
+  if (s->max_pages_per_seq < ceil_div(s->max_seqlen, s->page_size)) return COSA_ERR_INVALID_ARG;
+  if (s->total_qblocks < ceil_div(s->max_seqlen, s->block_size)) return COSA_ERR_INVALID_ARG;
+  if (s->max_seqlen > s->total_tokens) return COSA_ERR_INVALID_ARG;
+  // TMA row coordinates of the page pool are int32
+  if (static_cast<long>(s->num_pages) * s->num_kv_heads * s->page_size >= (1L << 31)) return COSA_ERR_UNSUPPORTED;
+  const int npow2 = next_pow2(ceil_div(s->max_seqlen, s->block_size));
+  if (score_smem_bytes(s->head_dim, proxy_group(*s), s->block_size / 16, npow2) > 200 * 1024)
+    return COSA_ERR_UNSUPPORTED;
+  return COSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct WsLayout {
+  size_t kq_off, ks_off, total;
+};
+
+WsLayout ws_layout(const cosa_shape_t& s) {
+  WsLayout w{};
+  w.kq_off = kStatusBytes;
+  const size_t kq_bytes = static_cast<size_t>(s.num_kv_heads) * s.total_qblocks * s.head_dim;
+  w.ks_off = align_up(w.kq_off + kq_bytes, 256);
+  w.total = align_up(w.ks_off + static_cast<size_t>(s.num_kv_heads) * s.total_qblocks * 4, 256);
+  return w;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle and 64-element (128-byte) inner boxes.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+              const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint32_t elem[3] = {1, 1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
+            strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace cosa
+
+using namespace cosa;
+
+extern "C" {
+
+const char* cosa_error_string(int code) {
+  switch (code) {
+    case COSA_OK: return "ok";
+    case COSA_ERR_INVALID_ARG: return "invalid argument";
+    case COSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case COSA_ERR_WORKSPACE: return "workspace too small";
+    case COSA_ERR_CUDA: return "CUDA error";
+    case COSA_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case COSA_ERR_DEVICE: return "device bounds check failed";
+    default: return "unknown status";
+  }
+}
+
+int cosa_version(void) { return 100; }
+
+void cosa_debug_set_wait_limit(uint32_t spins) { g_wait_limit.store(spins == 0 ? kDefaultWaitLimit : spins); }
+
+size_t cosa_workspace_size(const cosa_shape_t* shape, float budget, int32_t* kmax_out) {
+  if (check_shape(shape) != COSA_OK) return 0;
+  if (!(budget > 0.0f && budget <= 1.0f)) return 0;
+  if (kmax_out != nullptr)
+    *kmax_out = keep_count(ceil_div(shape->max_seqlen, shape->block_size), budget_bp(budget));
+  return ws_layout(*shape).total;
+}
+
+int cosa_workspace_init(void* workspace, size_t ws_bytes, cosa_stream_t stream) {
+  if (workspace == nullptr || ws_bytes < kStatusBytes) return COSA_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, kStatusBytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? COSA_OK
+             : COSA_ERR_CUDA;
+}
+
+int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, const int32_t* page_table, float budget,
+               int32_t kmax, int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags, void* workspace,
+               size_t ws_bytes, cosa_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc != COSA_OK) return rc;
+  if (q == nullptr || k_pages == nullptr || page_table == nullptr || order == nullptr || count == nullptr ||
+      n_hrm == nullptr || hrm_flags == nullptr || workspace == nullptr)
+    return COSA_ERR_INVALID_ARG;
+  if (!(budget > 0.0f && budget <= 1.0f)) return COSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return COSA_ERR_INVALID_ARG;
+  const int bp = budget_bp(budget);
+  if (kmax < keep_count(ceil_div(shape->max_seqlen, shape->block_size), bp)) return COSA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(*shape);
+  if (ws_bytes < w.total) return COSA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  Status* status = reinterpret_cast<Status*>(ws);
+
+  KPoolArgs ka{};
+  ka.k_pages = static_cast<const __nv_bfloat16*>(k_pages);
+  ka.page_table = page_table;
+  ka.cu_seqlens = shape->cu_seqlens;
+  ka.cu_qblocks = shape->cu_qblocks;
+  ka.kq = reinterpret_cast<int8_t*>(ws + w.kq_off);
+  ka.ks = reinterpret_cast<float*>(ws + w.ks_off);
+  ka.status = status;
+  ka.batch = shape->batch;
+  ka.num_kv_heads = shape->num_kv_heads;
+  ka.head_dim = shape->head_dim;
+  ka.block_size = shape->block_size;
+  ka.page_size = shape->page_size;
+  ka.max_pages_per_seq = shape->max_pages_per_seq;
+  ka.num_pages = shape->num_pages;
+  ka.nkb_total = shape->total_qblocks;
+  if (launch_kpool(ka, st) != cudaSuccess) return COSA_ERR_CUDA;
+
+  ScoreArgs sa{};
+  sa.q = static_cast<const __nv_bfloat16*>(q);
+  sa.kq = ka.kq;
+  sa.ks = ka.ks;
+  sa.cu_seqlens = shape->cu_seqlens;
+  sa.cu_qblocks = shape->cu_qblocks;
+  sa.order = order;
+  sa.count = count;
+  sa.n_hrm = n_hrm;
+  sa.hrm = hrm_flags;
+  sa.status = status;
+  sa.batch = shape->batch;
+  sa.num_q_heads = shape->num_q_heads;
+  sa.num_kv_heads = shape->num_kv_heads;
+  sa.head_dim = shape->head_dim;
+  sa.block_size = shape->block_size;
+  sa.nqb_total = shape->total_qblocks;
+  sa.kmax = kmax;
+  sa.bp = bp;
+  sa.npow2_max = next_pow2(ceil_div(shape->max_seqlen, shape->block_size));
+  if (launch_score(sa, proxy_group(*shape), st) != cudaSuccess) return COSA_ERR_CUDA;
+  return COSA_OK;
+}
+
+int cosa_remap(const cosa_shape_t* shape, const int32_t* page_table, const int32_t* order, const int32_t* count,
+               int32_t kmax, int32_t* pages, cosa_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc != COSA_OK) return rc;
+  if (page_table == nullptr || order == nullptr || count == nullptr || pages == nullptr || kmax < 1)
+    return COSA_ERR_INVALID_ARG;
+  RemapArgs ra{};
+  ra.page_table = page_table;
+  ra.order = order;
+  ra.count = count;
+  ra.cu_seqlens = shape->cu_seqlens;
+  ra.cu_qblocks = shape->cu_qblocks;
+  ra.pages = pages;
+  ra.status = nullptr;
+  ra.batch = shape->batch;
+  ra.num_q_heads = shape->num_q_heads;
+  ra.block_size = shape->block_size;
+  ra.page_size = shape->page_size;
+  ra.max_pages_per_seq = shape->max_pages_per_seq;
+  ra.num_pages = shape->num_pages;
+  ra.nqb_total = shape->total_qblocks;
+  ra.kmax = kmax;
+  return launch_remap(ra, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COSA_OK : COSA_ERR_CUDA;
+}
+
+int cosa_attn(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
+              const int32_t* page_table, const int32_t* order, const int32_t* count, int32_t kmax, float tau,
+              void* out, int32_t* visited, int32_t* skipped, uint8_t* skipbits, void* workspace, size_t ws_bytes,
+              cosa_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc != COSA_OK) return rc;
+  if (q == nullptr || k_pages == nullptr || v_pages == nullptr || page_table == nullptr || order == nullptr ||
+      count == nullptr || out == nullptr || visited == nullptr || skipped == nullptr || workspace == nullptr ||
+      kmax < 1)
+    return COSA_ERR_INVALID_ARG;
+  if (!(tau >= 0.0f && tau < 1.0f)) return COSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return COSA_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return COSA_ERR_WORKSPACE;
+
+  const int D = shape->head_dim;
+  const int Hq = shape->num_q_heads;
+  CUtensorMap qmap, kmap, vmap;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hq),
+                                static_cast<cuuint64_t>(shape->total_tokens)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hq) * D * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    if (!make_map(&qmap, q, 3, dims, strides, box)) return COSA_ERR_CUDA;
+  }
+  {
+    const cuuint64_t rows = static_cast<cuuint64_t>(shape->num_pages) * shape->num_kv_heads * shape->page_size;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(shape->page_size)};
+    if (!make_map(&kmap, k_pages, 2, dims, strides, box)) return COSA_ERR_CUDA;
+    if (!make_map(&vmap, v_pages, 2, dims, strides, box)) return COSA_ERR_CUDA;
+  }
+  OskArgs oa{};
+  oa.page_table = page_table;
+  oa.order = order;
+  oa.count = count;
+  oa.cu_seqlens = shape->cu_seqlens;
+  oa.cu_qblocks = shape->cu_qblocks;
+  oa.k_pages = static_cast<const __nv_bfloat16*>(k_pages);
+  oa.v_pages = static_cast<const __nv_bfloat16*>(v_pages);
+  oa.out = static_cast<__nv_bfloat16*>(out);
+  oa.visited = visited;
+  oa.skipped = skipped;
+  oa.skipbits = skipbits;
+  oa.status = reinterpret_cast<Status*>(workspace);
+  oa.batch = shape->batch;
+  oa.num_q_heads = Hq;
+  oa.num_kv_heads = shape->num_kv_heads;
+  oa.block_size = shape->block_size;
+  oa.page_size = shape->page_size;
+  oa.max_pages_per_seq = shape->max_pages_per_seq;
+  oa.num_pages = shape->num_pages;
+  oa.nqb_total = shape->total_qblocks;
+  oa.kmax = kmax;
+  oa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  oa.log2_tau = tau > 0.0f ? static_cast<float>(std::log2(static_cast<double>(tau))) : -INFINITY;
+  oa.wait_limit = g_wait_limit.load();
+  return launch_osk(oa, qmap, kmap, vmap, D, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COSA_OK
+                                                                                                      : COSA_ERR_CUDA;
+}
+
+int cosa_sync_status(void* workspace, cosa_stream_t stream) {
+  if (workspace == nullptr) return COSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Status h{};
+  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return COSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return COSA_ERR_CUDA;
+  if (h.bits == 0) return COSA_OK;
+  if (cudaMemsetAsync(workspace, 0, sizeof(h), st) != cudaSuccess) return COSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return COSA_ERR_CUDA;
+  return (h.bits & kErrTimeout) ? COSA_ERR_TIMEOUT : COSA_ERR_DEVICE;
+}
+
+}  // extern "C"

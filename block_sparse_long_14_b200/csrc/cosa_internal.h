@@ -1,0 +1,80 @@
+// Host-side argument blocks and launchers shared between libcosa's .cu files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "cosa.h"
+
+namespace cosa {
+
+struct Status;
+
+struct KPoolArgs {
+  const __nv_bfloat16* k_pages;
+  const int32_t* page_table;
+  const int32_t* cu_seqlens;
+  const int32_t* cu_qblocks;
+  int8_t* kq;     // [Hkv, NKB, d]
+  float* ks;      // [Hkv, NKB]
+  Status* status;
+  int batch, num_kv_heads, head_dim, block_size, page_size, max_pages_per_seq, num_pages, nkb_total;
+};
+
+struct ScoreArgs {
+  const __nv_bfloat16* q;
+  const int8_t* kq;
+  const float* ks;
+  const int32_t* cu_seqlens;
+  const int32_t* cu_qblocks;
+  int32_t* order;
+  int32_t* count;
+  int32_t* n_hrm;
+  uint8_t* hrm;
+  Status* status;
+  int batch, num_q_heads, num_kv_heads, head_dim, block_size, nqb_total, kmax, bp, npow2_max;
+};
+
+struct RemapArgs {
+  const int32_t* page_table;
+  const int32_t* order;
+  const int32_t* count;
+  const int32_t* cu_seqlens;
+  const int32_t* cu_qblocks;
+  int32_t* pages;
+  Status* status;
+  int batch, num_q_heads, block_size, page_size, max_pages_per_seq, num_pages, nqb_total, kmax;
+};
+
+struct OskArgs {
+  const int32_t* page_table;
+  const int32_t* order;
+  const int32_t* count;
+  const int32_t* cu_seqlens;
+  const int32_t* cu_qblocks;
+  const __nv_bfloat16* k_pages;
+  const __nv_bfloat16* v_pages;
+  __nv_bfloat16* out;
+  int32_t* visited;
+  int32_t* skipped;
+  uint8_t* skipbits;
+  Status* status;
+  int batch, num_q_heads, num_kv_heads, block_size, page_size, max_pages_per_seq, num_pages;
+  int nqb_total, kmax;
+  float scale_log2;  // log2(e) / sqrt(d)
+  float log2_tau;    // log2(tau), -inf for tau = 0
+  uint32_t wait_limit;
+};
+
+size_t score_smem_bytes(int D, int GT, int R, int npow2_max);
+cudaError_t launch_kpool(const KPoolArgs& a, cudaStream_t stream);
+cudaError_t launch_score(const ScoreArgs& a, int GT, cudaStream_t stream);
+cudaError_t launch_remap(const RemapArgs& a, cudaStream_t stream);
+cudaError_t launch_osk(const OskArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                       const CUtensorMap& vmap, int head_dim, cudaStream_t stream);
+size_t osk_smem_bytes(int head_dim, int block_size);
+
+}  // namespace cosa

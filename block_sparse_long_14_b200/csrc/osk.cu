@@ -1,0 +1,474 @@
+// Ordered-Skipping Kernel (OSK) for sm_100a.
+//
+// "CoSA: Accelerating Long-Context Inference via Proxy-Kernel Co-Designed
+// Sparse Attention":
+//   §4.3 "Physical jumping over pages" -- the inner loop runs only over the
+//        retained blocks; dropped blocks cost no iteration, no mask test and
+//        no synchronisation.
+//   §4.3 "In-kernel logic skip" -- after S = Q K^T of a visited block, the
+//        value side (exp, row sum, P V) is skipped when the block's row
+//        maxima are negligible against the running max; one vote per
+//        128-row query tile.
+//   §4.3 "Any-order page visiting" -- blocks are visited in the order KAP
+//        emitted (HRM first) through a page remap of the paged KV cache.
+//   §3.3 L1 -- QK^T is paid for every visited block; L2.1/L2.2 -- the test
+//        uses the running max and is an AND over the tile's rows.
+//   Appendix C.2 (Algorithm A) and D.1 (b = 128 logical blocks, pages of any
+//        size b_p resolving a block; the vote reuses the on-chip row maxima).
+//
+// One CTA per (query head, q-block) tile, 192 threads, warp-specialised:
+//   warps 0-3  softmax: one thread per query row.  tcgen05.ld of its S row
+//              from TMEM, causal mask, row max, the skip vote (warp __all_sync
+//              + a 4-warp named barrier), exp2 -> bf16 P into shared memory
+//              (128B-swizzled K-major, the UMMA operand layout), the row sum,
+//              lazy rescaling of O in TMEM, and the epilogue O / l -> bf16.
+//   warp 4     producer: page remap (order -> page_table) and TMA loads of the
+//              Q tile and of each block's K and V pages into a 2-stage ring;
+//              a block that ends past the sequence is copied by hand with
+//              zero fill so no stray page slot reaches an MMA.
+//   warp 5     MMA issuer: S = Q K^T (M=128, N=b, K=d) into one of two TMEM S
+//              buffers, then O += P V (M=128, N=d, K=b) unless the tile voted
+//              to skip; completion is signalled with tcgen05.commit.
+// S for block t+1 is computed while the softmax warps work on block t.
+// Every wait is bounded; on expiry the CTA records COSA_ERR_TIMEOUT, drains
+// its own copies and MMAs, frees TMEM and exits.
+#include <cstdint>
+#include <cmath>
+
+#include "cosa_device.cuh"
+#include "cosa_internal.h"
+
+namespace cosa {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBQ = 128;          // query rows per tile (TMEM lanes)
+constexpr uint32_t kDrainLimit = 1u << 22;
+constexpr float kRescaleLog2 = 8.0f;  // re-base O when the row max grows by > 2^8
+
+template <int D, int BK>
+struct Cfg {
+  static constexpr int Q_BYTES = kBQ * D * 2;
+  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int P_BYTES = kBQ * BK * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int TMEM_S0 = 0;
+  static constexpr int TMEM_S1 = BK;
+  static constexpr int TMEM_O = 2 * BK;
+  static constexpr int TMEM_NEED = 2 * BK + D;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                   : TMEM_NEED <= 256 ? 256 : 512;
+  // Shared memory is padded so that the CTAs resident on one SM never ask
+  // for more than the SM's 512 TMEM columns together (an allocation would
+  // otherwise wait for another CTA to finish).
+  static constexpr int SMEM_USED = OFF_BAR + 256 + 1024;  // barriers/flags + alignment slack
+  static constexpr int SMEM_MIN = TMEM_COLS == 512 ? 116 * 1024 : TMEM_COLS == 256 ? 78 * 1024 : 0;
+  static constexpr int SMEM = SMEM_USED > SMEM_MIN ? SMEM_USED : SMEM_MIN;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kBQ, BK, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBQ, D, false, true);
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort;
+  int skip_flag[2];
+  int vote[2][4];
+};
+
+// Copy one key block (K or V) of `nvalid` tokens into a 128B-swizzled stage
+// by hand, zero-filling rows past the sequence end or on a missing page.
+template <int D, int BK>
+__device__ void manual_block_copy(unsigned char* stage, const __nv_bfloat16* pool, const int32_t* pt_row,
+                                  int j, int nvalid, const OskArgs& a, int g, int lane) {
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  const int ppb = a.block_size / a.page_size;
+  for (int idx = lane; idx < BK * CH; idx += 32) {
+    const int row = idx / CH, ch = idx % CH;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (row < nvalid) {
+      const int page = __ldg(pt_row + j * ppb + row / a.page_size);
+      if (page >= 0 && page < a.num_pages) {
+        const __nv_bfloat16* src =
+            pool + ((static_cast<long>(page) * a.num_kv_heads + g) * a.page_size + row % a.page_size) * D + ch * 8;
+        v = __ldg(reinterpret_cast<const uint4*>(src));
+      } else {
+        report(a.status, kErrBounds, 0x300);
+      }
+    }
+    const int atom = ch >> 3, cc = ch & 7;
+    *reinterpret_cast<uint4*>(stage + atom * (BK * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+  }
+  fence_proxy_async();
+  __syncwarp();
+}
+
+}  // namespace
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+    osk_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+               const __grid_constant__ CUtensorMap vmap, const OskArgs a) {
+  using C = Cfg<D, BK>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = smem + C::OFF_Q;
+  unsigned char* sK = smem + C::OFF_K;
+  unsigned char* sV = smem + C::OFF_V;
+  unsigned char* sP = smem + C::OFF_P;
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  volatile int* abort = &bars->abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- tile: kv-head-major, longest rows first within a kv head
+  const int G = a.num_q_heads / a.num_kv_heads;
+  const int per_kv = G * a.nqb_total;
+  const int tile = blockIdx.x;
+  const int g = tile / per_kv;
+  const int rem = tile % per_kv;
+  const int I = a.nqb_total - 1 - rem / G;
+  const int h = g * G + rem % G;
+  const int s = find_seq(a.cu_qblocks, a.batch, I);
+  const int i = I - __ldg(a.cu_qblocks + s);
+  const int tok0 = __ldg(a.cu_seqlens + s);
+  const int L = __ldg(a.cu_seqlens + s + 1) - tok0;
+  const int b = a.block_size;
+  const int nrows = min(b, L - i * b);
+  const int nkb = (L + b - 1) / b;
+  const long row_id = static_cast<long>(h) * a.nqb_total + I;
+  int n = __ldg(a.count + row_id);
+  if (n < 0 || n > a.kmax) {
+    if (tid == 0) report(a.status, kErrBounds, 0x301);
+    n = n < 0 ? 0 : a.kmax;
+  }
+  const int32_t* ord = a.order + row_id * a.kmax;
+  const int32_t* pt_row = a.page_table + static_cast<long>(s) * a.max_pages_per_seq;
+
+  if (tid == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->k_full[x], 1);
+      mbar_init(&bars->k_empty[x], 1);
+      mbar_init(&bars->v_full[x], 1);
+      mbar_init(&bars->v_empty[x], 1);
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->s_free[x], kBQ);
+      mbar_init(&bars->p_full[x], kBQ);
+    }
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->mma_drain, 1);
+    bars->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (n == 0) {
+    // nothing listed: zero rows, zero counts
+    if (warp < 4 && tid < nrows) {
+      uint4* dst = reinterpret_cast<uint4*>(a.out + ((static_cast<long>(tok0) + i * b + tid) * a.num_q_heads + h) * D);
+      for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (tid == 0) { a.visited[row_id] = 0; a.skipped[row_id] = 0; }
+    if (a.skipbits != nullptr && tid < a.kmax) a.skipbits[row_id * a.kmax + tid] = 0;
+  } else if (warp == 4) {
+    // =========================================================== producer
+    int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1};
+    bool ok = true;
+    if (lane == 0) {
+      prefetch_tmap(&qmap);
+      prefetch_tmap(&kmap);
+      prefetch_tmap(&vmap);
+      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * (kBQ * 128), &qmap, &bars->q_full, c * 64, h, tok0 + i * b);
+    }
+    const int ppb = b / a.page_size;
+    for (int t = 0; t < n && ok; ++t) {
+      const int slot = t & 1, use = t >> 1;
+      int j = __ldg(ord + t);
+      bool jvalid = (j >= 0 && j < nkb);
+      if (!jvalid) {
+        if (lane == 0) report(a.status, kErrBounds, 0x302);
+        j = 0;
+      }
+      const int nvalid = jvalid ? min(b, L - j * b) : 0;
+      // Page ids of the block (lane u holds page u); a bad id sends the block down the checked path.
+      int page = -1;
+      if (lane < ppb && jvalid && j * b + lane * a.page_size < L) page = __ldg(pt_row + j * ppb + lane);
+      const bool pages_ok = __all_sync(0xffffffffu, lane >= ppb || (page >= 0 && page < a.num_pages));
+      const bool via_tma = jvalid && nvalid == b && pages_ok;
+      for (int kvsel = 0; kvsel < 2 && ok; ++kvsel) {
+        uint64_t* full = kvsel == 0 ? &bars->k_full[slot] : &bars->v_full[slot];
+        uint64_t* empty = kvsel == 0 ? &bars->k_empty[slot] : &bars->v_empty[slot];
+        unsigned char* stage = (kvsel == 0 ? sK : sV) + slot * C::KV_BYTES;
+        const CUtensorMap* map = kvsel == 0 ? &kmap : &vmap;
+        if (use >= 1 && lane == 0) ok = mbar_wait(empty, (use - 1) & 1, a.wait_limit, abort, a.status, 0x10 + kvsel);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (via_tma) {
+          if (lane == 0) mbar_arrive_expect_tx(full, C::KV_BYTES);
+          for (int u = 0; u < ppb; ++u) {
+            const int pg = __shfl_sync(0xffffffffu, page, u);
+            if (lane == 0) {
+              const int row = (pg * a.num_kv_heads + g) * a.page_size;
+#pragma unroll
+              for (int c = 0; c < D / 64; ++c)
+                tma_load_2d(stage + c * (BK * 128) + u * a.page_size * 128, map, full, c * 64, row);
+            }
+          }
+          __syncwarp();
+        } else {
+          manual_block_copy<D, BK>(stage, kvsel == 0 ? a.k_pages : a.v_pages, pt_row, j, nvalid, a, g, lane);
+          if (lane == 0) mbar_arrive(full);
+        }
+        if (kvsel == 0) k_armed[slot] = use; else v_armed[slot] = use;
+      }
+    }
+    // drain: every load this warp started has landed before the CTA exits
+    if (lane == 0) {
+      mbar_wait(&bars->q_full, 0, kDrainLimit, abort, nullptr, 0);
+      for (int x = 0; x < 2; ++x) {
+        if (k_armed[x] >= 0) mbar_wait(&bars->k_full[x], k_armed[x] & 1, kDrainLimit, abort, nullptr, 0);
+        if (v_armed[x] >= 0) mbar_wait(&bars->v_full[x], v_armed[x] & 1, kDrainLimit, abort, nullptr, 0);
+      }
+    }
+  } else if (warp == 5) {
+    // =========================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
+      bool ok = mbar_wait(&bars->q_full, 0, a.wait_limit, abort, a.status, 0x20);
+      bool first_pv = true;
+      for (int t = 0; t <= n && ok; ++t) {
+        if (t < n) {
+          const int slot = t & 1, use = t >> 1;
+          ok = mbar_wait(&bars->k_full[slot], use & 1, a.wait_limit, abort, a.status, 0x21);
+          if (ok && t >= 2) ok = mbar_wait(&bars->s_free[slot], (use - 1) & 1, a.wait_limit, abort, a.status, 0x22);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t d_s = tmem + (slot ? C::TMEM_S1 : C::TMEM_S0);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ad = sw128_desc(q_base + (ks >> 2) * (kBQ * 128) + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(k_base + slot * C::KV_BYTES + (ks >> 2) * (BK * 128) + (ks & 3) * 32, 16, 1024);
+            tc_mma_ss(d_s, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars->s_full[slot]);
+          tc_commit(&bars->k_empty[slot]);
+        }
+        if (t >= 1) {
+          const int u = t - 1, vslot = u & 1, vuse = u >> 1;
+          ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, a.wait_limit, abort, a.status, 0x23);
+          if (ok) ok = mbar_wait(&bars->v_full[vslot], vuse & 1, a.wait_limit, abort, a.status, 0x24);
+          if (!ok) break;
+          tc_fence_after();
+          const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[u & 1]);
+          if (!skip) {
+            const uint32_t d_o = tmem + C::TMEM_O;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = sw128_desc(p_base + (kk >> 2) * (kBQ * 128) + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(v_base + vslot * C::KV_BYTES + kk * 2048, BK * 128, 1024);
+              tc_mma_ss(d_o, ad, bd, C::IDESC_PV, (!first_pv || kk > 0) ? 1u : 0u);
+            }
+            first_pv = false;
+            tc_commit(&bars->v_empty[vslot]);
+            tc_commit(&bars->o_done);
+          } else {
+            mbar_arrive(&bars->v_empty[vslot]);
+          }
+        }
+      }
+      // drain: all MMAs issued by this thread complete before TMEM is freed
+      tc_commit(&bars->mma_drain);
+      mbar_wait(&bars->mma_drain, 0, kDrainLimit, abort, nullptr, 0);
+    }
+    __syncwarp();
+  } else {
+    // =========================================================== softmax (warps 0-3)
+    const int r = tid;  // tile row = TMEM lane
+    const bool row_valid = r < nrows;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m = -INFINITY, mref = -INFINITY, l = 0.0f;
+    int n_pv = 0, nskip = 0;
+    bool aborted = false;
+    for (int t = 0; t < n; ++t) {
+      const int sb = t & 1;
+      bool ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, a.wait_limit, abort, a.status, 0x30);
+      ok = __all_sync(0xffffffffu, ok) && !aborted;
+      float sv[BK];
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) tmem_ld32(lane_base + (sb ? C::TMEM_S1 : C::TMEM_S0) + c * 32, sv + c * 32);
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[sb]);
+      }
+      // causal mask: key k of block j is visible to row r iff j*b + k <= i*b + r
+      const int j = __ldg(ord + t);
+      const int lim = r - (j - i) * b;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < BK; ++k) {
+        if (k > lim) sv[k] = -INFINITY;
+        mx = fmaxf(mx, sv[k]);
+      }
+      const float m_blk = (row_valid && mx != -INFINITY) ? mx * a.scale_log2 : -INFINITY;
+      const float gap = (m_blk == -INFINITY) ? -INFINITY : m_blk - m;
+      const bool votes_skip = !row_valid || gap < a.log2_tau;
+      const bool wskip = __all_sync(0xffffffffu, votes_skip);
+      if (lane == 0) bars->vote[sb][warp] = (ok ? 0 : 2) | (wskip ? 1 : 0);
+      named_bar_sync(1, 4 * 32);
+      const int v0 = bars->vote[sb][0], v1 = bars->vote[sb][1], v2 = bars->vote[sb][2], v3 = bars->vote[sb][3];
+      if ((v0 | v1 | v2 | v3) & 2) { aborted = true; break; }
+      const bool skip = (v0 & v1 & v2 & v3) & 1;
+      if (skip) {
+        if (r == 0) {
+          bars->skip_flag[sb] = 1;
+          ++nskip;
+          if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 1;
+        }
+        mbar_arrive(&bars->p_full[sb]);
+        continue;
+      }
+      const float m_new = fmaxf(m, m_blk);
+      if (n_pv >= 1) {
+        bool okw = mbar_wait(&bars->o_done, (n_pv - 1) & 1, a.wait_limit, abort, a.status, 0x31);
+        if (!__all_sync(0xffffffffu, okw)) { aborted = true; continue; }
+        tc_fence_after();
+        const bool need = row_valid && (m_new > mref + kRescaleLog2);
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = row_valid ? ex2_approx(mref - m_new) : 1.0f;
+          l *= alpha;
+          if (row_valid) mref = m_new;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tmem_ld32(lane_base + C::TMEM_O + c * 32, ov);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(lane_base + C::TMEM_O + c * 32, ov);
+          }
+          tc_wait_st();
+        }
+      } else if (row_valid) {
+        mref = m_new;
+      }
+      m = m_new;
+      // P = exp2(s * log2e/sqrt(d) - mref) in bf16, written in the UMMA K-major SW128 layout
+      const float nb = -mref;
+      float lsum = 0.0f;
+#pragma unroll
+      for (int c8 = 0; c8 < BK / 8; ++c8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float p0 = 0.0f, p1 = 0.0f;
+          if (row_valid) {
+            p0 = ex2_approx(fmaf(sv[c8 * 8 + 2 * e], a.scale_log2, nb));
+            p1 = ex2_approx(fmaf(sv[c8 * 8 + 2 * e + 1], a.scale_log2, nb));
+          }
+          pk[e] = pack_bf16x2(p0, p1);
+          lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+        }
+        const int atom = c8 >> 3, cc = c8 & 7;
+        *reinterpret_cast<uint4*>(sP + atom * (kBQ * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l += lsum;
+      fence_proxy_async();
+      tc_fence_before();
+      if (r == 0) {
+        bars->skip_flag[sb] = 0;
+        if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 0;
+      }
+      mbar_arrive(&bars->p_full[sb]);
+      ++n_pv;
+    }
+    // ---- epilogue: O / l -> bf16
+    bool ok = !aborted && n_pv >= 1;
+    if (ok) ok = mbar_wait(&bars->o_done, (n_pv - 1) & 1, a.wait_limit, abort, a.status, 0x32);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = (row_valid && l > 0.0f) ? 1.0f / l : 0.0f;
+      __nv_bfloat16* dst = a.out + ((static_cast<long>(tok0) + i * b + r) * a.num_q_heads + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float ov[32];
+        tmem_ld32(lane_base + C::TMEM_O + c * 32, ov);
+        tc_wait_ld();
+        if (row_valid) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 w4;
+            w4.x = pack_bf16x2(ov[q4 * 8 + 0] * inv_l, ov[q4 * 8 + 1] * inv_l);
+            w4.y = pack_bf16x2(ov[q4 * 8 + 2] * inv_l, ov[q4 * 8 + 3] * inv_l);
+            w4.z = pack_bf16x2(ov[q4 * 8 + 4] * inv_l, ov[q4 * 8 + 5] * inv_l);
+            w4.w = pack_bf16x2(ov[q4 * 8 + 6] * inv_l, ov[q4 * 8 + 7] * inv_l);
+            *reinterpret_cast<uint4*>(dst + c * 32 + q4 * 8) = w4;
+          }
+        }
+      }
+    }
+    if (r == 0) {
+      a.visited[row_id] = n;
+      a.skipped[row_id] = nskip;
+      if (a.skipbits != nullptr)
+        for (int t = n; t < a.kmax; ++t) a.skipbits[row_id * a.kmax + t] = 0;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+template <int D, int BK>
+static cudaError_t launch_t(const OskArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                            const CUtensorMap& vmap, cudaStream_t stream) {
+  using C = Cfg<D, BK>;
+  auto kern = osk_kernel<D, BK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(a.num_q_heads) * a.nqb_total;
+  kern<<<grid, kThreads, C::SMEM, stream>>>(qmap, kmap, vmap, a);
+  return cudaGetLastError();
+}
+
+size_t osk_smem_bytes(int head_dim, int block_size) {
+  if (head_dim == 128) return block_size == 128 ? Cfg<128, 128>::SMEM : Cfg<128, 64>::SMEM;
+  return block_size == 128 ? Cfg<64, 128>::SMEM : Cfg<64, 64>::SMEM;
+}
+
+cudaError_t launch_osk(const OskArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                       int head_dim, cudaStream_t stream) {
+  if (head_dim == 128)
+    return a.block_size == 128 ? launch_t<128, 128>(a, qmap, kmap, vmap, stream)
+                               : launch_t<128, 64>(a, qmap, kmap, vmap, stream);
+  return a.block_size == 128 ? launch_t<64, 128>(a, qmap, kmap, vmap, stream)
+                             : launch_t<64, 64>(a, qmap, kmap, vmap, stream);
+}
+
+}  // namespace cosa

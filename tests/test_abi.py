@@ -1,0 +1,108 @@
+"""The C ABI library on the host (no GPU needed): it builds for sm_100a, loads,
+exports every entry point include/cosa.h declares, and its host-side logic
+(argument checks, workspace sizing, list length kmax) behaves as declared.
+No call here launches a kernel.
+"""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import block_sparse_long_14_b200 as cosa
+from block_sparse_long_14_b200 import build as cbuild
+from oracle import kap
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cosa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    cbuild.build()
+    return cosa.lib()
+
+
+def declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"COSA_API\s+[\w\s\*]+?\b(cosa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared()
+    for n in ("cosa_proxy", "cosa_remap", "cosa_attn", "cosa_workspace_size", "cosa_sync_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", cosa.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (cosa_\w+)", out))
+    assert set(declared()) <= exported
+    for n in declared():
+        assert hasattr(lib, n)
+
+
+def test_library_is_built_for_sm100a(lib):
+    out = subprocess.run(["cuobjdump", "--list-elf", cosa.LIB_PATH], capture_output=True, text=True)
+    if out.returncode == 0:
+        assert "sm_100a" in out.stdout
+
+
+def test_error_strings(lib):
+    for code in range(7):
+        assert lib.cosa_error_string(code)
+    assert lib.cosa_version() >= 100
+
+
+def _shape(**kw):
+    base = dict(batch=1, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=128, page_size=64,
+                num_pages=2048, max_pages_per_seq=2048, total_tokens=131072, total_qblocks=1024,
+                max_seqlen=131072, cu_seqlens=16, cu_qblocks=32)   # pointers are not dereferenced here
+    base.update(kw)
+    return cosa._Shape(**base)
+
+
+def _ws(shape, budget):
+    k = ctypes.c_int32(0)
+    n = cosa.lib().cosa_workspace_size(ctypes.byref(shape), ctypes.c_float(budget), ctypes.byref(k))
+    return n, k.value
+
+
+@pytest.mark.parametrize("budget", [0.05, 0.1, 0.2, 0.25, 1.0])
+@pytest.mark.parametrize("max_seqlen,b", [(131072, 128), (90000, 128), (1024, 64), (1, 128)])
+def test_workspace_size_and_kmax(lib, budget, max_seqlen, b):
+    nqb = (max_seqlen + b - 1) // b
+    sh = _shape(block_size=b, max_seqlen=max_seqlen, total_tokens=max_seqlen, total_qblocks=nqb,
+                max_pages_per_seq=(max_seqlen + 63) // 64)
+    n, kmax = _ws(sh, budget)
+    assert kmax == kap.kmax_for(nqb, budget)
+    assert n >= 256 + 8 * nqb * 128 + 8 * nqb * 4 and n % 256 == 0
+
+
+@pytest.mark.parametrize("bad", [
+    dict(head_dim=96), dict(block_size=256), dict(page_size=48), dict(page_size=4), dict(num_kv_heads=5),
+    dict(num_q_heads=64, num_kv_heads=4), dict(max_pages_per_seq=10), dict(cu_seqlens=0), dict(batch=0),
+    dict(total_qblocks=3),
+])
+def test_invalid_shapes_are_rejected(lib, bad):
+    assert _ws(_shape(**bad), 0.1)[0] == 0
+
+
+def test_invalid_budgets_are_rejected(lib):
+    for b in (0.0, -0.1, 1.5, float("nan")):
+        assert _ws(_shape(), b)[0] == 0
+
+
+def test_null_pointers_rejected_before_launch(lib):
+    sh = _shape()
+    rc = lib.cosa_proxy(ctypes.byref(sh), None, None, None, ctypes.c_float(0.1), 64, None, None, None, None, None,
+                        0, None)
+    assert rc == 1
+    rc = lib.cosa_attn(ctypes.byref(sh), None, None, None, None, None, None, 52, ctypes.c_float(1e-4), None, None,
+                       None, None, None, 0, None)
+    assert rc == 1
+    rc = lib.cosa_remap(ctypes.byref(sh), None, None, None, 52, None, None)
+    assert rc == 1

@@ -1,0 +1,132 @@
+"""GPU parity: libcosa (through its C ABI) vs the CPU oracle, element by element.
+
+Small packed batches that finish in seconds on the oracle yet span several
+tiles, ragged tails, partial pages, several page sizes, head_dim 64/128,
+block size 64/128 and GQA groups 1/4/8.
+"""
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_14_b200 as cosa
+from oracle import dense, kap, osk
+from synth import make_custom, make_workload
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": lambda: make_workload(1),
+    "ragged_b128_p64": lambda: make_custom([1000, 300, 2100, 129], 8, 2, 128, 128, 64, structure="llama", seed=21),
+    "ragged_b128_p16_g1": lambda: make_custom([700, 1500], 4, 4, 128, 128, 16, structure="llama", seed=22),
+    "d64_b128_p32": lambda: make_custom([1200, 513], 4, 2, 64, 128, 32, structure="llama", seed=23),
+    "b64_g8": lambda: make_custom([900, 200], 16, 2, 128, 64, 64, structure="llama", seed=24),
+    "short_seqs": lambda: make_custom([50, 128, 1, 129], 4, 1, 128, 128, 64, structure="random", seed=25),
+    "qwen_mix": lambda: make_custom([1500], 32, 8, 128, 128, 64, structure="qwen", seed=26),
+}
+
+
+@functools.lru_cache(maxsize=None)
+def workload(name):
+    return CASES[name]()
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_proxy(name, budget):
+    w = workload(name)
+    return kap.kap_proxy(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, budget)
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_attn(name, budget, tau):
+    w = workload(name)
+    r = oracle_proxy(name, budget)
+    return osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size,
+                   r["order"], r["count"], tau)
+
+
+@functools.lru_cache(maxsize=None)
+def device(name):
+    return gu.upload(workload(name))
+
+
+@pytest.mark.parametrize("budget", [0.25, 1.0, 0.05])
+@pytest.mark.parametrize("name", list(CASES))
+def test_proxy_bit_exact(name, budget):
+    got, kmax, _ = gu.run_proxy(device(name), budget)
+    ref = oracle_proxy(name, budget)
+    assert kmax == ref["kmax"]
+    gu.assert_proxy_equal(got, ref)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_remap_bit_exact(name):
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], 0.25, kmax, ws)
+    pages = cosa.remap(d["batch"], d["page_table"], sel["order"], sel["count"], kmax)
+    cosa.check(ws)
+    ref = oracle_proxy(name, 0.25)
+    expect = kap.remap(ref["order"], ref["count"], w.page_table, w.seqlens, w.block_size, w.page_size)
+    assert np.array_equal(pages.cpu().numpy(), expect)
+
+
+@pytest.mark.parametrize("budget,tau", [(0.25, 1e-4), (0.25, 0.0), (1.0, 1e-2), (0.25, 1e-2)])
+@pytest.mark.parametrize("name", list(CASES))
+def test_attn_matches_oracle(name, budget, tau):
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], budget)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], budget, kmax, ws)
+    res = gu.run_attn(d, sel, kmax, tau, ws)
+    ref = oracle_attn(name, budget, tau)
+    stats = gu.compare_attn(res, ref, w, tau, gu.all_units(w))
+    if tau == 0.0:
+        assert int(res["skipped"].sum()) == 0
+    print(name, budget, tau, stats)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_b128_p64", "b64_g8"])
+def test_full_budget_no_skip_equals_dense(name):
+    """Budget 100% and tau = 0: OSK is dense causal attention (fp64 brute force)."""
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], 1.0)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], 1.0, kmax, ws)
+    res = gu.run_attn(d, sel, kmax, 0.0, ws)
+    ref = dense.dense_causal(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads)
+    err = np.abs(res["out"].float().cpu().numpy() - ref)
+    assert err.max() <= gu.MAX_ABS and err.mean() <= gu.MEAN_ABS
+
+
+def test_order_invariance_on_gpu():
+    """tau = 0: a random permutation of every visit list changes only rounding."""
+    name = "ragged_b128_p64"
+    d = device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], 0.25, kmax, ws)
+    a = gu.run_attn(d, sel, kmax, 0.0, ws)["out"].float()
+    order = sel["order"].clone()
+    cnt = sel["count"].cpu().numpy()
+    o = order.cpu().numpy()
+    rng = np.random.default_rng(3)
+    for h in range(o.shape[0]):
+        for I in range(o.shape[1]):
+            o[h, I, :cnt[h, I]] = rng.permutation(o[h, I, :cnt[h, I]])
+    perm = torch.from_numpy(o).cuda()
+    b = gu.run_attn(d, dict(order=perm, count=sel["count"]), kmax, 0.0, ws)["out"].float()
+    assert (a - b).abs().max().item() <= gu.MAX_ABS
+    assert (a - b).abs().mean().item() <= gu.MEAN_ABS
+
+
+def test_repeated_calls_are_deterministic():
+    d = device("qwen_mix")
+    ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
+    outs = []
+    for _ in range(3):
+        sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], 0.25, kmax, ws)
+        r = gu.run_attn(d, sel, kmax, 1e-4, ws)
+        outs.append((sel["order"].clone(), r["out"].clone(), r["skipped"].clone()))
+    for o in outs[1:]:
+        assert torch.equal(o[0], outs[0][0]) and torch.equal(o[1], outs[0][1]) and torch.equal(o[2], outs[0][2])
