@@ -72,33 +72,44 @@ def workload_config(w):
     return {"workload": w.name, "seq_len": max(w.seqlens), "batch": w.batch, "num_q_heads": w.num_q_heads,
             "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
             "page_size": w.page_size, "pages": "shuffled pool" if w.meta.get("shuffled_pages") else "contiguous",
-            "budget": BUDGET, "tau": TAU,
+            "budget": w.budgets[0], "tau": TAU,
             "l2": "inputs larger than L2 (q 1 GiB + k/v pages 512 MiB per step), no flush"}
 
 
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
+    """nvidia-smi samples (every 50 ms, timestamped) kept only inside the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(1.5)   # let the sampler come up before the timed region
         except OSError:
             self.proc = None
-        return self
 
-    def __exit__(self, *exc):
-        self.lines = []
+    def begin(self):
+        import datetime
+        self.t0 = datetime.datetime.now()
+
+    def end(self):
+        import datetime
+        self.t1 = datetime.datetime.now()
+
+    def stop(self):
         if self.proc is not None:
+            time.sleep(0.2)
             self.proc.terminate()
             try:
                 out, _ = self.proc.communicate(timeout=5)
@@ -108,23 +119,28 @@ class Clocks:
             self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        import datetime
+        sm, mx, power, reasons = [], None, [], set()
+        for l in self.lines:
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                if self.t0 is not None and not (self.t0 <= ts <= self.t1):
+                    continue
+                sm.append(float(f[2]))
+                mx = float(f[3])
+                power.append(float(f[4]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.REASONS, f[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
 
 
 # ------------------------------------------------------------------ CPU side
@@ -208,7 +224,8 @@ def run_cosa(args, rank, world, local_rank):
     w = make_workload(args.config, seed=rank_seed(args.config, rank, world))
     d = upload(w)
     batch = d["batch"]
-    ws, kmax = cosa.alloc_workspace(batch, BUDGET)
+    budget = w.budgets[0]
+    ws, kmax = cosa.alloc_workspace(batch, budget)
     H, N = w.num_q_heads, batch.total_qblocks
     sel = dict(order=torch.empty((H, N, kmax), dtype=torch.int32, device="cuda"),
                count=torch.empty((H, N), dtype=torch.int32, device="cuda"),
@@ -221,7 +238,7 @@ def run_cosa(args, rank, world, local_rank):
     def step(tau=TAU, ev=None):
         if ev is not None:
             ev[0].record(stream)
-        cosa.proxy(batch, d["q"], d["k_pages"], d["page_table"], BUDGET, kmax, ws, out=sel)
+        cosa.proxy(batch, d["q"], d["k_pages"], d["page_table"], budget, kmax, ws, out=sel)
         if ev is not None:
             ev[1].record(stream)
         cosa.attn(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], sel["order"], sel["count"], kmax,
@@ -229,6 +246,8 @@ def run_cosa(args, rank, world, local_rank):
         if ev is not None:
             ev[2].record(stream)
 
+    clk = Clocks(local_rank)
+    clk.start()
     for _ in range(max(3, args.warmup)):
         step()
     cosa.check(ws)
@@ -238,12 +257,14 @@ def run_cosa(args, rank, world, local_rank):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    with Clocks(local_rank) as clk:
-        start.record(stream)
-        for k in range(args.steps):
-            step(ev=evs[k])
-        stop.record(stream)
-        torch.cuda.synchronize()
+    clk.begin()
+    start.record(stream)
+    for k in range(args.steps):
+        step(ev=evs[k])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    clk.end()
+    clk.stop()
     if dist is not None:
         dist.barrier()
     cosa.check(ws)
@@ -412,8 +433,8 @@ def run_cosa(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cosa", choices=["cosa", "reference"])
     ap.add_argument("--config", type=int, default=CONFIG_ID)
     ap.add_argument("--quick", action="store_true", help="skip the tau sweep, dense reference and e2e legs")

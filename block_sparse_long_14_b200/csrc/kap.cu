@@ -133,7 +133,7 @@ __device__ __forceinline__ bool better(float s2, int j2, float s1, int j1) {
 // Threads: 256.  GT = query heads per CTA (all sharing one kv head),
 // R = sub-rows of 16 rows per q-block.
 template <int D, int GT, int R>
-__global__ void __launch_bounds__(256) kap_score_select_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(256, 2) kap_score_select_kernel(ScoreArgs a) {
   constexpr int COLS = GT * D;
   constexpr int NCHUNK = COLS / 8;       // 16-byte chunks per token row of the head group
   constexpr int QB = D / 4;              // bytes of a row each MMA quad-lane owns
