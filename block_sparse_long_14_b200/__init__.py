@@ -54,6 +54,8 @@ _SIGS = {
     "cosa_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "cosa_proxy": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, ctypes.c_float, ctypes.c_int32,
                                   _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "cosa_proxy_noalloc": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, ctypes.c_float, ctypes.c_int32,
+                                          _P, _P, _P, _P, _P]),
     "cosa_remap": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, ctypes.c_int32, _P, _P]),
     "cosa_attn": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_float,
                                  _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -160,6 +162,30 @@ def proxy(batch: Batch, q, k_pages, page_table, budget: float, kmax: int, worksp
                            _ptr(out["n_hrm"], torch.int32, "n_hrm"), _ptr(out["hrm"], torch.uint8, "hrm"),
                            _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream())
     _check(rc, "cosa_proxy")
+    return out
+
+
+def proxy_noalloc(batch: Batch, q, k_pages, page_table, budget: float, kmax: int, out=None):
+    """KAP without a workspace, for callers that cannot allocate device memory.
+
+    The pooled keys go to the library's fixed static device scratch array
+    instead (see cosa_proxy_noalloc in include/cosa.h for its size limit and
+    its sharing rules).  The output lists are still the caller's: pass them
+    in `out` to avoid any allocation here.
+    """
+    H, N = batch.num_q_heads, batch.total_qblocks
+    dev = q.device
+    if out is None:
+        out = dict(order=torch.empty((H, N, kmax), dtype=torch.int32, device=dev),
+                   count=torch.empty((H, N), dtype=torch.int32, device=dev),
+                   n_hrm=torch.empty((H, N), dtype=torch.int32, device=dev),
+                   hrm=torch.empty((H, N, kmax), dtype=torch.uint8, device=dev))
+    rc = _lib().cosa_proxy_noalloc(ctypes.byref(batch.c), _ptr(q, torch.bfloat16, "q"),
+                                   _ptr(k_pages, torch.bfloat16, "k_pages"), _ptr(page_table, torch.int32, "page_table"),
+                                   ctypes.c_float(budget), int(kmax), _ptr(out["order"], torch.int32, "order"),
+                                   _ptr(out["count"], torch.int32, "count"), _ptr(out["n_hrm"], torch.int32, "n_hrm"),
+                                   _ptr(out["hrm"], torch.uint8, "hrm"), _stream())
+    _check(rc, "cosa_proxy_noalloc")
     return out
 
 

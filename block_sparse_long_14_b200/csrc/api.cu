@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "cosa_device.cuh"
 #include "cosa_internal.h"
@@ -304,3 +305,94 @@ int cosa_sync_status(void* workspace, cosa_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// cosa_proxy_noalloc: the proxy with its pooled-key scratch in a static device
+// array instead of a caller-provided workspace (contract in include/cosa.h).
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[COSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side name is only a stand-in for the symbol).
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return COSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return COSA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return COSA_OK;
+}
+}  // namespace
+
+extern "C" int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, const void* k_pages,
+                                  const int32_t* page_table, float budget, int32_t kmax, int32_t* order,
+                                  int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags, cosa_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc != COSA_OK) return rc;
+  if (q == nullptr || k_pages == nullptr || page_table == nullptr || order == nullptr || count == nullptr ||
+      n_hrm == nullptr || hrm_flags == nullptr)
+    return COSA_ERR_INVALID_ARG;
+  if (!(budget > 0.0f && budget <= 1.0f)) return COSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages)) return COSA_ERR_INVALID_ARG;
+  const int bp = budget_bp(budget);
+  if (kmax < keep_count(ceil_div(shape->max_seqlen, shape->block_size), bp)) return COSA_ERR_INVALID_ARG;
+  // pooled keys [Hkv, NQB, d] int8, then scales [Hkv, NQB] fp32
+  const size_t kq_bytes = align_up(static_cast<size_t>(shape->num_kv_heads) * shape->total_qblocks * shape->head_dim, 256);
+  const size_t need = kq_bytes + static_cast<size_t>(shape->num_kv_heads) * shape->total_qblocks * 4;
+  if (need > COSA_NOALLOC_SCRATCH_BYTES) return COSA_ERR_WORKSPACE;
+  void* base = nullptr;
+  rc = noalloc_scratch(&base);
+  if (rc != COSA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* scratch = static_cast<unsigned char*>(base);
+
+  KPoolArgs ka{};
+  ka.k_pages = static_cast<const __nv_bfloat16*>(k_pages);
+  ka.page_table = page_table;
+  ka.cu_seqlens = shape->cu_seqlens;
+  ka.cu_qblocks = shape->cu_qblocks;
+  ka.kq = reinterpret_cast<int8_t*>(scratch);
+  ka.ks = reinterpret_cast<float*>(scratch + kq_bytes);
+  ka.status = nullptr;
+  ka.batch = shape->batch;
+  ka.num_kv_heads = shape->num_kv_heads;
+  ka.head_dim = shape->head_dim;
+  ka.block_size = shape->block_size;
+  ka.page_size = shape->page_size;
+  ka.max_pages_per_seq = shape->max_pages_per_seq;
+  ka.num_pages = shape->num_pages;
+  ka.nkb_total = shape->total_qblocks;
+  if (launch_kpool(ka, st) != cudaSuccess) return COSA_ERR_CUDA;
+
+  ScoreArgs sa{};
+  sa.q = static_cast<const __nv_bfloat16*>(q);
+  sa.kq = ka.kq;
+  sa.ks = ka.ks;
+  sa.cu_seqlens = shape->cu_seqlens;
+  sa.cu_qblocks = shape->cu_qblocks;
+  sa.order = order;
+  sa.count = count;
+  sa.n_hrm = n_hrm;
+  sa.hrm = hrm_flags;
+  sa.status = nullptr;
+  sa.batch = shape->batch;
+  sa.num_q_heads = shape->num_q_heads;
+  sa.num_kv_heads = shape->num_kv_heads;
+  sa.head_dim = shape->head_dim;
+  sa.block_size = shape->block_size;
+  sa.nqb_total = shape->total_qblocks;
+  sa.kmax = kmax;
+  sa.bp = bp;
+  sa.npow2_max = next_pow2(ceil_div(shape->max_seqlen, shape->block_size));
+  if (launch_score(sa, proxy_group(*shape), st) != cudaSuccess) return COSA_ERR_CUDA;
+  return COSA_OK;
+}

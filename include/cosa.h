@@ -144,6 +144,38 @@ COSA_API int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_
                int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags,
                void* workspace, size_t ws_bytes, cosa_stream_t stream);
 
+/* Capacity of the static device scratch array behind cosa_proxy_noalloc. */
+#define COSA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * cosa_proxy for callers that cannot allocate device memory.  (The paper has
+ * no counterpart: this is a library convenience, not part of the method.)
+ *
+ * Who needs it: code that runs inside an inference engine which has already
+ * reserved nearly all device memory for its own pools (a serving framework's
+ * KV cache) and offers no scratch API, and code on a latency-critical path
+ * where cudaMalloc, which can fail under such a reservation and can
+ * synchronise the device, is not acceptable.
+ *
+ * Same arguments and outputs as cosa_proxy, minus the workspace.  The pooled
+ * key scratch lives instead in one static device array of
+ * COSA_NOALLOC_SCRATCH_BYTES bytes that every GPU loading this library holds
+ * until the process exits.  Limit: shapes whose pooled keys need more
+ * (num_kv_heads * total_qblocks * (head_dim + 4) bytes, plus alignment) are
+ * rejected with COSA_ERR_WORKSPACE before anything is enqueued.
+ *
+ * The first call on a device (with that device current) looks up the array's
+ * device address; make that first call before any stream capture.  The call
+ * allocates nothing and frees nothing.  Every call shares the one array and
+ * overwrites it completely, so calls that overlap on the GPU (for example on
+ * two streams) race; serialise them.  Device-side bounds checks still skip a
+ * bad access but, without a workspace status word, are not reported.
+ */
+COSA_API int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, const void* k_pages,
+                                const int32_t* page_table, float budget, int32_t kmax,
+                                int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags,
+                                cosa_stream_t stream);
+
 /*
  * Page remap (§4.3 "Any-order page visiting"): ordered key blocks -> pages.
  *   pages  device int32 [Hq, NQB, kmax * (b / b_p)]:
