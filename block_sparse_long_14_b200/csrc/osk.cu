@@ -16,20 +16,26 @@
 //   Appendix C.2 (Algorithm A) and D.1 (b = 128 logical blocks, pages of any
 //        size b_p resolving a block; the vote reuses the on-chip row maxima).
 //
-// One CTA per (query head, q-block) tile, 192 threads, warp-specialised:
-//   warps 0-3  softmax: one thread per query row.  tcgen05.ld of its S row
-//              from TMEM, causal mask, row max, the skip vote (warp __all_sync
-//              + a 4-warp named barrier), exp2 -> bf16 P into shared memory
-//              (128B-swizzled K-major, the UMMA operand layout), the row sum,
-//              lazy rescaling of O in TMEM, and the epilogue O / l -> bf16.
-//   warp 4     producer: page remap (order -> page_table) and TMA loads of the
-//              Q tile and of each block's K and V pages into a 2-stage ring;
-//              a block that ends past the sequence is copied by hand with
-//              zero fill so no stray page slot reaches an MMA.
-//   warp 5     MMA issuer: S = Q K^T (M=128, N=b, K=d) into one of two TMEM S
-//              buffers, then O += P V (M=128, N=d, K=b) unless the tile voted
-//              to skip; completion is signalled with tcgen05.commit.
-// S for block t+1 is computed while the softmax warps work on block t.
+// One CTA per (query head, q-block) tile, 320 threads, warp-specialised:
+//   warps 0-7  softmax: two threads per query row (TMEM lane), each owning
+//              half of the block's key columns.  tcgen05.ld of its half row,
+//              causal mask on the diagonal block, half-row max, the skip vote
+//              (a row votes to skip iff both of its halves lie below the
+//              threshold, so no exchange is needed: warp __all_sync + one
+//              256-thread named barrier), exp2 -> bf16 P into one of two
+//              shared-memory P buffers (128B-swizzled K-major, the UMMA
+//              operand layout), partial row sums, lazy rescaling of its half
+//              of O in TMEM, and the epilogue O / l -> bf16.
+//   warp 8     producer: page remap (order -> page_table) and TMA loads of the
+//              Q tile and of each block's K and V pages into 2-stage rings; a
+//              block ending past the sequence is copied by hand with zero
+//              fill so no stray page slot reaches an MMA.
+//   warp 9     MMA issuer: S = Q K^T (M=128, N=b, K=d) into one of two TMEM S
+//              buffers, then O += P V (M=128, N=d, K=b) from the P buffer of
+//              that kept block, unless the tile voted to skip; completion is
+//              signalled with tcgen05.commit.
+// S for block t+1 is computed while the softmax warps work on block t, and
+// with two P buffers the softmax of block t does not wait for P V of t-1.
 // Every wait is bounded; on expiry the CTA records COSA_ERR_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
 #include <cstdint>
@@ -42,7 +48,11 @@ namespace cosa {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kBQ = 128;          // query rows per tile (TMEM lanes)
 constexpr uint32_t kDrainLimit = 1u << 22;
 constexpr float kRescaleLog2 = 8.0f;  // re-base O when the row max grows by > 2^8
@@ -56,7 +66,8 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
   static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int HALF = BK / 2;   // key columns per softmax thread
   static constexpr int TMEM_S0 = 0;
   static constexpr int TMEM_S1 = BK;
   static constexpr int TMEM_O = 2 * BK;
@@ -66,11 +77,12 @@ struct Cfg {
   // Shared memory is padded so that the CTAs resident on one SM never ask
   // for more than the SM's 512 TMEM columns together (an allocation would
   // otherwise wait for another CTA to finish).
-  static constexpr int SMEM_USED = OFF_BAR + 256 + 1024;  // barriers/flags + alignment slack
+  static constexpr int SMEM_USED = OFF_BAR + 2304;  // barriers, flags and the half-row exchange
   static constexpr int SMEM_MIN = TMEM_COLS == 512 ? 116 * 1024 : TMEM_COLS == 256 ? 78 * 1024 : 0;
   static constexpr int SMEM = SMEM_USED > SMEM_MIN ? SMEM_USED : SMEM_MIN;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kBQ, BK, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBQ, D, false, true);
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
 struct Bars {
@@ -78,13 +90,16 @@ struct Bars {
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t p_full[2];   // softmax verdict (and P, if kept) for block t, by t & 1
+  uint64_t p_free[2];   // P V of the kept block using P buffer x has completed
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
   int skip_flag[2];
-  int vote[2][4];
+  int vote[2][kSoftmaxWarps];
+  int vote_end[kSoftmaxWarps];
+  float half_max[2][2][kBQ];   // [t & 1][half][row]: exchange of half-row maxima;
+                               // the epilogue reuses slot [n & 1] for partial row sums
 };
 
 // Copy one key block (K or V) of `nvalid` tokens into a 128B-swizzled stage
@@ -121,8 +136,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     osk_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const OskArgs a) {
   using C = Cfg<D, BK>;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) unsigned char smem[];
+  // The operand tiles need 1024-byte alignment for the 128B swizzle; dynamic
+  // shared memory starts right after the CTA's reserved 1 KiB, which gives it.
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) report(a.status, kErrBounds, 0x3FF);
+    return;
+  }
   unsigned char* sQ = smem + C::OFF_Q;
   unsigned char* sK = smem + C::OFF_K;
   unsigned char* sV = smem + C::OFF_V;
@@ -164,15 +184,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_full[x], 1);
       mbar_init(&bars->v_empty[x], 1);
       mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->s_free[x], kBQ);
-      mbar_init(&bars->p_full[x], kBQ);
+      mbar_init(&bars->s_free[x], kSoftmaxThreads);
+      mbar_init(&bars->p_full[x], kSoftmaxThreads);
+      mbar_init(&bars->p_free[x], 1);
     }
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->mma_drain, 1);
     bars->abort = 0;
     mbar_fence_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -183,13 +203,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (n == 0) {
     // nothing listed: zero rows, zero counts
-    if (warp < 4 && tid < nrows) {
+    if (tid < nrows) {
       uint4* dst = reinterpret_cast<uint4*>(a.out + ((static_cast<long>(tok0) + i * b + tid) * a.num_q_heads + h) * D);
       for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (tid == 0) { a.visited[row_id] = 0; a.skipped[row_id] = 0; }
     if (a.skipbits != nullptr && tid < a.kmax) a.skipbits[row_id * a.kmax + tid] = 0;
-  } else if (warp == 4) {
+  } else if (warp == kProducerWarp) {
     // =========================================================== producer
     int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1};
     bool ok = true;
@@ -251,12 +271,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (v_armed[x] >= 0) mbar_wait(&bars->v_full[x], v_armed[x] & 1, kDrainLimit, abort, nullptr, 0);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // =========================================================== MMA issuer
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
       bool ok = mbar_wait(&bars->q_full, 0, a.wait_limit, abort, a.status, 0x20);
-      bool first_pv = true;
+      int kept = 0;
       for (int t = 0; t <= n && ok; ++t) {
         if (t < n) {
           const int slot = t & 1, use = t >> 1;
@@ -282,16 +302,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[u & 1]);
           if (!skip) {
+            const int pb = kept & 1;
             const uint32_t d_o = tmem + C::TMEM_O;
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = sw128_desc(p_base + (kk >> 2) * (kBQ * 128) + (kk & 3) * 32, 16, 1024);
+              const uint64_t ad =
+                  sw128_desc(p_base + pb * C::P_BYTES + (kk >> 2) * (kBQ * 128) + (kk & 3) * 32, 16, 1024);
               const uint64_t bd = sw128_desc(v_base + vslot * C::KV_BYTES + kk * 2048, BK * 128, 1024);
-              tc_mma_ss(d_o, ad, bd, C::IDESC_PV, (!first_pv || kk > 0) ? 1u : 0u);
+              tc_mma_ss(d_o, ad, bd, C::IDESC_PV, (kept > 0 || kk > 0) ? 1u : 0u);
             }
-            first_pv = false;
+            ++kept;
             tc_commit(&bars->v_empty[vslot]);
-            tc_commit(&bars->o_done);
+            tc_commit(&bars->p_free[pb]);
           } else {
             mbar_arrive(&bars->v_empty[vslot]);
           }
@@ -303,46 +325,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // =========================================================== softmax (warps 0-3)
-    const int r = tid;  // tile row = TMEM lane
+    // =========================================================== softmax (warps 0-7)
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;                 // tile row = TMEM lane
+    const int col0 = half * C::HALF;                // first key column of this thread
     const bool row_valid = r < nrows;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float sl2 = a.scale_log2;
     float m = -INFINITY, mref = -INFINITY, l = 0.0f;
     int n_pv = 0, nskip = 0;
     bool aborted = false;
+    int j_next = __ldg(ord);
     for (int t = 0; t < n; ++t) {
       const int sb = t & 1;
+      const int j = j_next;
+      if (t + 1 < n) j_next = __ldg(ord + t + 1);
       bool ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, a.wait_limit, abort, a.status, 0x30);
       ok = __all_sync(0xffffffffu, ok) && !aborted;
-      float sv[BK];
+      float sv[C::HALF];
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < BK / 32; ++c) tmem_ld32(lane_base + (sb ? C::TMEM_S1 : C::TMEM_S0) + c * 32, sv + c * 32);
+        for (int c = 0; c < C::HALF / 32; ++c)
+          tmem_ld32(lane_base + (sb ? C::TMEM_S1 : C::TMEM_S0) + col0 + c * 32, sv + c * 32);
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->s_free[sb]);
       }
-      // causal mask: key k of block j is visible to row r iff j*b + k <= i*b + r
-      const int j = __ldg(ord + t);
-      const int lim = r - (j - i) * b;
-      float mx = -INFINITY;
+      // causal mask (only the diagonal block, or a block past it, can hide keys):
+      // key k of block j is visible to row r iff j*b + k <= i*b + r
+      if (j >= i) {
+        const int lim = r - (j - i) * b - col0;
 #pragma unroll
-      for (int k = 0; k < BK; ++k) {
-        if (k > lim) sv[k] = -INFINITY;
-        mx = fmaxf(mx, sv[k]);
+        for (int k = 0; k < C::HALF; ++k)
+          if (k > lim) sv[k] = -INFINITY;
       }
-      const float m_blk = (row_valid && mx != -INFINITY) ? mx * a.scale_log2 : -INFINITY;
-      const float gap = (m_blk == -INFINITY) ? -INFINITY : m_blk - m;
+      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+      for (int k = 4; k < C::HALF; k += 4) {
+        mx0 = fmaxf(mx0, sv[k]);
+        mx1 = fmaxf(mx1, sv[k + 1]);
+        mx2 = fmaxf(mx2, sv[k + 2]);
+        mx3 = fmaxf(mx3, sv[k + 3]);
+      }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      const float m_half = (row_valid && mx != -INFINITY) ? mx * sl2 : -INFINITY;
+      const float gap = (m_half == -INFINITY) ? -INFINITY : m_half - m;
       const bool votes_skip = !row_valid || gap < a.log2_tau;
       const bool wskip = __all_sync(0xffffffffu, votes_skip);
       if (lane == 0) bars->vote[sb][warp] = (ok ? 0 : 2) | (wskip ? 1 : 0);
-      named_bar_sync(1, 4 * 32);
-      const int v0 = bars->vote[sb][0], v1 = bars->vote[sb][1], v2 = bars->vote[sb][2], v3 = bars->vote[sb][3];
-      if ((v0 | v1 | v2 | v3) & 2) { aborted = true; break; }
-      const bool skip = (v0 & v1 & v2 & v3) & 1;
-      if (skip) {
-        if (r == 0) {
+      bars->half_max[sb][half][r] = m_half;
+      named_bar_sync(1, kSoftmaxThreads);
+      int vor = 0, vand = 1;
+#pragma unroll
+      for (int w = 0; w < kSoftmaxWarps; ++w) {
+        const int v = bars->vote[sb][w];
+        vor |= v;
+        vand &= v;
+      }
+      if (vor & 2) { aborted = true; break; }
+      if (vand & 1) {
+        if (tid == 0) {
           bars->skip_flag[sb] = 1;
           ++nskip;
           if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 1;
@@ -350,55 +393,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars->p_full[sb]);
         continue;
       }
-      const float m_new = fmaxf(m, m_blk);
-      if (n_pv >= 1) {
-        bool okw = mbar_wait(&bars->o_done, (n_pv - 1) & 1, a.wait_limit, abort, a.status, 0x31);
+      const float m_row = fmaxf(m_half, bars->half_max[sb][half ^ 1][r]);
+      const float m_new = fmaxf(m, m_row);
+      // the reference max of P / l / O: re-based lazily (identical in both halves of a row)
+      float new_ref = mref;
+      bool rescale = false;
+      if (n_pv == 0) {
+        if (row_valid) new_ref = m_new;
+      } else {
+        const bool need = row_valid && (m_new > mref + kRescaleLog2);
+        rescale = __any_sync(0xffffffffu, need);
+        if (rescale && row_valid) new_ref = m_new;
+      }
+      // P = exp2(s * log2e/sqrt(d) - ref) in bf16; partial row sum of the rounded values
+      uint32_t pk[C::HALF / 2];
+      float ls0 = 0.0f, ls1 = 0.0f;
+      const float nb = (new_ref == -INFINITY) ? 0.0f : -new_ref;
+#pragma unroll
+      for (int e = 0; e < C::HALF / 2; ++e) {
+        const float p0 = ex2_approx(fmaf(sv[2 * e], sl2, nb));
+        const float p1 = ex2_approx(fmaf(sv[2 * e + 1], sl2, nb));
+        pk[e] = row_valid ? pack_bf16x2(p0, p1) : 0u;
+        ls0 += __uint_as_float(pk[e] << 16);
+        ls1 += __uint_as_float(pk[e] & 0xFFFF0000u);
+      }
+      if (rescale) {
+        // O must be complete up to the last kept block before it is re-based
+        bool okw = mbar_wait(&bars->p_free[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status,
+                             0x31);
         if (!__all_sync(0xffffffffu, okw)) { aborted = true; continue; }
         tc_fence_after();
-        const bool need = row_valid && (m_new > mref + kRescaleLog2);
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = row_valid ? ex2_approx(mref - m_new) : 1.0f;
-          l *= alpha;
-          if (row_valid) mref = m_new;
+        const float alpha = row_valid ? ex2_approx(mref - new_ref) : 1.0f;
+        l *= alpha;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float ov[32];
-            tmem_ld32(lane_base + C::TMEM_O + c * 32, ov);
-            tc_wait_ld();
+        for (int c = 0; c < D / 64; ++c) {
+          float ov[32];
+          const uint32_t addr = lane_base + C::TMEM_O + half * (D / 2) + c * 32;
+          tmem_ld32(addr, ov);
+          tc_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-            tmem_st32(lane_base + C::TMEM_O + c * 32, ov);
-          }
-          tc_wait_st();
+          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+          tmem_st32(addr, ov);
         }
-      } else if (row_valid) {
-        mref = m_new;
+        tc_wait_st();
       }
+      mref = new_ref;
       m = m_new;
-      // P = exp2(s * log2e/sqrt(d) - mref) in bf16, written in the UMMA K-major SW128 layout
-      const float nb = -mref;
-      float lsum = 0.0f;
-#pragma unroll
-      for (int c8 = 0; c8 < BK / 8; ++c8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float p0 = 0.0f, p1 = 0.0f;
-          if (row_valid) {
-            p0 = ex2_approx(fmaf(sv[c8 * 8 + 2 * e], a.scale_log2, nb));
-            p1 = ex2_approx(fmaf(sv[c8 * 8 + 2 * e + 1], a.scale_log2, nb));
-          }
-          pk[e] = pack_bf16x2(p0, p1);
-          lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
-        }
-        const int atom = c8 >> 3, cc = c8 & 7;
-        *reinterpret_cast<uint4*>(sP + atom * (kBQ * 128) + r * 128 + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      l += ls0 + ls1;
+      // P buffer of this kept block: free once P V of the kept block two back has completed
+      const int pb = n_pv & 1;
+      if (n_pv >= 2) {
+        bool okw = mbar_wait(&bars->p_free[pb], ((n_pv >> 1) - 1) & 1, a.wait_limit, abort, a.status, 0x33);
+        if (!__all_sync(0xffffffffu, okw)) { aborted = true; continue; }
       }
-      l += lsum;
+      unsigned char* prow = sP + pb * C::P_BYTES + r * 128;
+#pragma unroll
+      for (int c8 = 0; c8 < C::HALF / 8; ++c8) {
+        const int chunk = col0 / 8 + c8;          // 16-byte chunk index along the keys
+        const int atom = chunk >> 3, cc = chunk & 7;
+        *reinterpret_cast<uint4*>(prow + atom * (kBQ * 128) + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+      }
       fence_proxy_async();
       tc_fence_before();
-      if (r == 0) {
+      if (tid == 0) {
         bars->skip_flag[sb] = 0;
         if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 0;
       }
@@ -407,16 +465,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- epilogue: O / l -> bf16
     bool ok = !aborted && n_pv >= 1;
-    if (ok) ok = mbar_wait(&bars->o_done, (n_pv - 1) & 1, a.wait_limit, abort, a.status, 0x32);
+    if (ok) ok = mbar_wait(&bars->p_free[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status, 0x32);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    float (*half_l)[kBQ] = bars->half_max[n & 1];   // idle since the barrier of block n-1
+    half_l[half][r] = l;
+    if (lane == 0) bars->vote_end[warp] = ok ? 1 : 0;
+    named_bar_sync(1, kSoftmaxThreads);
+    int all_ok = 1;
+#pragma unroll
+    for (int w = 0; w < kSoftmaxWarps; ++w) all_ok &= bars->vote_end[w];
+    if (all_ok) {
       tc_fence_after();
-      const float inv_l = (row_valid && l > 0.0f) ? 1.0f / l : 0.0f;
-      __nv_bfloat16* dst = a.out + ((static_cast<long>(tok0) + i * b + r) * a.num_q_heads + h) * D;
+      const float lrow = half_l[0][r] + half_l[1][r];
+      const float inv_l = (row_valid && lrow > 0.0f) ? 1.0f / lrow : 0.0f;
+      __nv_bfloat16* dst = a.out + ((static_cast<long>(tok0) + i * b + r) * a.num_q_heads + h) * D + half * (D / 2);
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         float ov[32];
-        tmem_ld32(lane_base + C::TMEM_O + c * 32, ov);
+        tmem_ld32(lane_base + C::TMEM_O + half * (D / 2) + c * 32, ov);
         tc_wait_ld();
         if (row_valid) {
 #pragma unroll
@@ -431,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (r == 0) {
+    if (tid == 0) {
       a.visited[row_id] = n;
       a.skipped[row_id] = nskip;
       if (a.skipbits != nullptr)
@@ -442,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 template <int D, int BK>
