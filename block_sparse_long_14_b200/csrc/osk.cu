@@ -22,20 +22,20 @@
 //              causal mask on the diagonal block, half-row max, the skip vote
 //              (a row votes to skip iff both of its halves lie below the
 //              threshold, so no exchange is needed: warp __all_sync + one
-//              256-thread named barrier), exp2 -> bf16 P into one of two
-//              shared-memory P buffers (128B-swizzled K-major, the UMMA
-//              operand layout), partial row sums, lazy rescaling of its half
-//              of O in TMEM, and the epilogue O / l -> bf16.
+//              256-thread named barrier), exp2 -> bf16 P written back into
+//              its own half of the S columns in TMEM, partial row sums, lazy
+//              rescaling of its half of O in TMEM, the epilogue O / l.
 //   warp 8     producer: page remap (order -> page_table) and TMA loads of the
-//              Q tile and of each block's K and V pages into 2-stage rings; a
+//              Q tile and of each block's K and V pages into 3-stage rings; a
 //              block ending past the sequence is copied by hand with zero
 //              fill so no stray page slot reaches an MMA.
-//   warp 9     MMA issuer: S = Q K^T (M=128, N=b, K=d) into one of two TMEM S
-//              buffers, then O += P V (M=128, N=d, K=b) from the P buffer of
-//              that kept block, unless the tile voted to skip; completion is
-//              signalled with tcgen05.commit.
-// S for block t+1 is computed while the softmax warps work on block t, and
-// with two P buffers the softmax of block t does not wait for P V of t-1.
+//   warp 9     MMA issuer: S = Q K^T (M=128, N=b, K=d; both operands in shared
+//              memory) into one of two TMEM S buffers, then O += P V
+//              (M=128, N=d, K=b) with P read from TMEM, unless the tile voted
+//              to skip; completion is signalled with tcgen05.commit.
+// The tensor pipe executes one thread's MMAs in issue order, so P V of block
+// t-2 has read its P before S of block t overwrites the same columns; S for
+// block t+1 is computed while the softmax warps work on block t.
 // Every wait is bounded; on expiry the CTA records COSA_ERR_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
 #include <cstdint>
@@ -54,20 +54,37 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr int kBQ = 128;          // query rows per tile (TMEM lanes)
+constexpr int kStages = 3;        // K and V ring depth
 constexpr uint32_t kDrainLimit = 1u << 22;
 constexpr float kRescaleLog2 = 8.0f;  // re-base O when the row max grows by > 2^8
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];   // softmax verdict (and P, if kept) for block t, by t & 1
+  uint64_t o_done[2];   // P V of kept block c has completed, by c & 1
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort;
+  int skip_flag[2];
+  int vote[2][kSoftmaxWarps];
+  int vote_end[kSoftmaxWarps];
+  float half_max[2][2][kBQ];   // [t & 1][half][row]: exchange of half-row maxima;
+                               // the epilogue reuses slot [n & 1] for partial row sums
+};
 
 template <int D, int BK>
 struct Cfg {
   static constexpr int Q_BYTES = kBQ * D * 2;
   static constexpr int KV_BYTES = BK * D * 2;
-  static constexpr int P_BYTES = kBQ * BK * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_V = OFF_K + kStages * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + kStages * KV_BYTES;
   static constexpr int HALF = BK / 2;   // key columns per softmax thread
+  static constexpr int KPH = HALF / 16; // K=16 MMA steps per half
   static constexpr int TMEM_S0 = 0;
   static constexpr int TMEM_S1 = BK;
   static constexpr int TMEM_O = 2 * BK;
@@ -77,29 +94,14 @@ struct Cfg {
   // Shared memory is padded so that the CTAs resident on one SM never ask
   // for more than the SM's 512 TMEM columns together (an allocation would
   // otherwise wait for another CTA to finish).
-  static constexpr int SMEM_USED = OFF_BAR + 2304;  // barriers, flags and the half-row exchange
+  static constexpr int SMEM_USED = OFF_BAR + static_cast<int>(sizeof(Bars));
   static constexpr int SMEM_MIN = TMEM_COLS == 512 ? 116 * 1024 : TMEM_COLS == 256 ? 78 * 1024 : 0;
   static constexpr int SMEM = SMEM_USED > SMEM_MIN ? SMEM_USED : SMEM_MIN;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(kBQ, BK, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBQ, D, false, true);
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
-};
-
-struct Bars {
-  uint64_t q_full;
-  uint64_t k_full[2], k_empty[2];
-  uint64_t v_full[2], v_empty[2];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2];   // softmax verdict (and P, if kept) for block t, by t & 1
-  uint64_t p_free[2];   // P V of the kept block using P buffer x has completed
-  uint64_t mma_drain;
-  uint32_t tmem_base;
-  int abort;
-  int skip_flag[2];
-  int vote[2][kSoftmaxWarps];
-  int vote_end[kSoftmaxWarps];
-  float half_max[2][2][kBQ];   // [t & 1][half][row]: exchange of half-row maxima;
-                               // the epilogue reuses slot [n & 1] for partial row sums
+  static_assert(OFF_BAR + sizeof(Bars) <= static_cast<size_t>(SMEM), "barrier block inside the allocation");
+  static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
 };
 
 // Copy one key block (K or V) of `nvalid` tokens into a 128B-swizzled stage
@@ -131,6 +133,8 @@ __device__ void manual_block_copy(unsigned char* stage, const __nv_bfloat16* poo
 
 }  // namespace
 
+// 10 warps put 3 warps on some SM sub-partitions, each with 16K registers,
+// which caps a thread at 168 registers.
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
     osk_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -146,7 +150,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sQ = smem + C::OFF_Q;
   unsigned char* sK = smem + C::OFF_K;
   unsigned char* sV = smem + C::OFF_V;
-  unsigned char* sP = smem + C::OFF_P;
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   volatile int* abort = &bars->abort;
 
@@ -178,15 +181,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < kStages; ++x) {
       mbar_init(&bars->k_full[x], 1);
       mbar_init(&bars->k_empty[x], 1);
       mbar_init(&bars->v_full[x], 1);
       mbar_init(&bars->v_empty[x], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->s_free[x], kSoftmaxThreads);
       mbar_init(&bars->p_full[x], kSoftmaxThreads);
-      mbar_init(&bars->p_free[x], 1);
+      mbar_init(&bars->o_done[x], 1);
     }
     mbar_init(&bars->mma_drain, 1);
     bars->abort = 0;
@@ -211,7 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (a.skipbits != nullptr && tid < a.kmax) a.skipbits[row_id * a.kmax + tid] = 0;
   } else if (warp == kProducerWarp) {
     // =========================================================== producer
-    int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1};
+    int k_armed[kStages], v_armed[kStages];
+    for (int x = 0; x < kStages; ++x) k_armed[x] = v_armed[x] = -1;
     bool ok = true;
     if (lane == 0) {
       prefetch_tmap(&qmap);
@@ -223,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int ppb = b / a.page_size;
     for (int t = 0; t < n && ok; ++t) {
-      const int slot = t & 1, use = t >> 1;
+      const int slot = t % kStages, use = t / kStages;
       int j = __ldg(ord + t);
       bool jvalid = (j >= 0 && j < nkb);
       if (!jvalid) {
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // drain: every load this warp started has landed before the CTA exits
     if (lane == 0) {
       mbar_wait(&bars->q_full, 0, kDrainLimit, abort, nullptr, 0);
-      for (int x = 0; x < 2; ++x) {
+      for (int x = 0; x < kStages; ++x) {
         if (k_armed[x] >= 0) mbar_wait(&bars->k_full[x], k_armed[x] & 1, kDrainLimit, abort, nullptr, 0);
         if (v_armed[x] >= 0) mbar_wait(&bars->v_full[x], v_armed[x] & 1, kDrainLimit, abort, nullptr, 0);
       }
@@ -274,46 +279,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // =========================================================== MMA issuer
     if (lane == 0) {
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
       bool ok = mbar_wait(&bars->q_full, 0, a.wait_limit, abort, a.status, 0x20);
       int kept = 0;
       for (int t = 0; t <= n && ok; ++t) {
         if (t < n) {
-          const int slot = t & 1, use = t >> 1;
+          const int slot = t % kStages, use = t / kStages;
           ok = mbar_wait(&bars->k_full[slot], use & 1, a.wait_limit, abort, a.status, 0x21);
-          if (ok && t >= 2) ok = mbar_wait(&bars->s_free[slot], (use - 1) & 1, a.wait_limit, abort, a.status, 0x22);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t d_s = tmem + (slot ? C::TMEM_S1 : C::TMEM_S0);
+          const uint32_t d_s = tmem + ((t & 1) ? C::TMEM_S1 : C::TMEM_S0);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint64_t ad = sw128_desc(q_base + (ks >> 2) * (kBQ * 128) + (ks & 3) * 32, 16, 1024);
             const uint64_t bd = sw128_desc(k_base + slot * C::KV_BYTES + (ks >> 2) * (BK * 128) + (ks & 3) * 32, 16, 1024);
             tc_mma_ss(d_s, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
           }
-          tc_commit(&bars->s_full[slot]);
+          tc_commit(&bars->s_full[t & 1]);
           tc_commit(&bars->k_empty[slot]);
         }
         if (t >= 1) {
-          const int u = t - 1, vslot = u & 1, vuse = u >> 1;
+          const int u = t - 1, vslot = u % kStages, vuse = u / kStages;
           ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, a.wait_limit, abort, a.status, 0x23);
           if (ok) ok = mbar_wait(&bars->v_full[vslot], vuse & 1, a.wait_limit, abort, a.status, 0x24);
           if (!ok) break;
           tc_fence_after();
           const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[u & 1]);
           if (!skip) {
-            const int pb = kept & 1;
+            const uint32_t p_tmem = tmem + ((u & 1) ? C::TMEM_S1 : C::TMEM_S0);
             const uint32_t d_o = tmem + C::TMEM_O;
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad =
-                  sw128_desc(p_base + pb * C::P_BYTES + (kk >> 2) * (kBQ * 128) + (kk & 3) * 32, 16, 1024);
+              // P of keys [16kk, 16kk+16): half kk / KPH wrote its P into the first
+              // HALF/2 columns of its own S half
+              const uint32_t a_t = p_tmem + (kk / C::KPH) * C::HALF + (kk % C::KPH) * 8;
               const uint64_t bd = sw128_desc(v_base + vslot * C::KV_BYTES + kk * 2048, BK * 128, 1024);
-              tc_mma_ss(d_o, ad, bd, C::IDESC_PV, (kept > 0 || kk > 0) ? 1u : 0u);
+              tc_mma_ts(d_o, a_t, bd, C::IDESC_PV, (kept > 0 || kk > 0) ? 1u : 0u);
             }
-            ++kept;
             tc_commit(&bars->v_empty[vslot]);
-            tc_commit(&bars->p_free[pb]);
+            tc_commit(&bars->o_done[kept & 1]);
+            ++kept;
           } else {
             mbar_arrive(&bars->v_empty[vslot]);
           }
@@ -338,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int j_next = __ldg(ord);
     for (int t = 0; t < n; ++t) {
       const int sb = t & 1;
+      const uint32_t s_cols = lane_base + (sb ? C::TMEM_S1 : C::TMEM_S0) + col0;
       const int j = j_next;
       if (t + 1 < n) j_next = __ldg(ord + t + 1);
       bool ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, a.wait_limit, abort, a.status, 0x30);
@@ -346,11 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < C::HALF / 32; ++c)
-          tmem_ld32(lane_base + (sb ? C::TMEM_S1 : C::TMEM_S0) + col0 + c * 32, sv + c * 32);
+        for (int c = 0; c < C::HALF / 32; ++c) tmem_ld32(s_cols + c * 32, sv + c * 32);
         tc_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&bars->s_free[sb]);
       }
       // causal mask (only the diagonal block, or a block past it, can hide keys):
       // key k of block j is visible to row r iff j*b + k <= i*b + r
@@ -390,6 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++nskip;
           if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 1;
         }
+        tc_fence_before();
         mbar_arrive(&bars->p_full[sb]);
         continue;
       }
@@ -419,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (rescale) {
         // O must be complete up to the last kept block before it is re-based
-        bool okw = mbar_wait(&bars->p_free[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status,
+        bool okw = mbar_wait(&bars->o_done[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status,
                              0x31);
         if (!__all_sync(0xffffffffu, okw)) { aborted = true; continue; }
         tc_fence_after();
@@ -435,26 +439,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e) ov[e] *= alpha;
           tmem_st32(addr, ov);
         }
-        tc_wait_st();
       }
       mref = new_ref;
       m = m_new;
       l += ls0 + ls1;
-      // P buffer of this kept block: free once P V of the kept block two back has completed
-      const int pb = n_pv & 1;
-      if (n_pv >= 2) {
-        bool okw = mbar_wait(&bars->p_free[pb], ((n_pv >> 1) - 1) & 1, a.wait_limit, abort, a.status, 0x33);
-        if (!__all_sync(0xffffffffu, okw)) { aborted = true; continue; }
+      // P over this thread's own (already read) S columns, packed bf16 pairs
+      if constexpr (C::HALF == 64) {
+        tmem_st32(s_cols, reinterpret_cast<const float*>(pk));
+      } else {
+        tmem_st16(s_cols, pk);
       }
-      unsigned char* prow = sP + pb * C::P_BYTES + r * 128;
-#pragma unroll
-      for (int c8 = 0; c8 < C::HALF / 8; ++c8) {
-        const int chunk = col0 / 8 + c8;          // 16-byte chunk index along the keys
-        const int atom = chunk >> 3, cc = chunk & 7;
-        *reinterpret_cast<uint4*>(prow + atom * (kBQ * 128) + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
-      }
-      fence_proxy_async();
+      tc_wait_st();
       tc_fence_before();
       if (tid == 0) {
         bars->skip_flag[sb] = 0;
@@ -465,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- epilogue: O / l -> bf16
     bool ok = !aborted && n_pv >= 1;
-    if (ok) ok = mbar_wait(&bars->p_free[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status, 0x32);
+    if (ok) ok = mbar_wait(&bars->o_done[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status, 0x32);
     ok = __all_sync(0xffffffffu, ok);
     float (*half_l)[kBQ] = bars->half_max[n & 1];   // idle since the barrier of block n-1
     half_l[half][r] = l;
