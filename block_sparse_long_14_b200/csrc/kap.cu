@@ -130,6 +130,30 @@ __device__ __forceinline__ bool better(float s2, int j2, float s1, int j1) {
   return s2 > s1 || (s2 == s1 && j2 < j1);
 }
 
+// Ascending bitonic sort of `nseg` independent segments of `size` keys
+// (a power of two), segment x at base + x * stride.  Whole-CTA (256 threads);
+// index arithmetic by shifts and masks.
+__device__ void bitonic_sort(uint64_t* base, int nseg, int size, int stride) {
+  if (size < 2) return;
+  int lg_n = 0;
+  while ((1 << lg_n) < size) ++lg_n;
+  const int pairs = nseg * size / 2;
+  for (int k = 2, lg_k = 1; k <= size; k <<= 1, ++lg_k) {
+    for (int jj = k >> 1, lg_j = lg_k - 1; jj > 0; jj >>= 1, --lg_j) {
+      for (int idx = threadIdx.x; idx < pairs; idx += blockDim.x) {
+        const int seg = idx >> (lg_n - 1);
+        const int li = idx & ((size >> 1) - 1);
+        const int x = ((li >> lg_j) << (lg_j + 1)) | (li & (jj - 1));
+        uint64_t* p = base + seg * stride;
+        const uint64_t va = p[x], vb = p[x + jj];
+        const bool asc = (x & k) == 0;
+        if ((va > vb) == asc) { p[x] = vb; p[x + jj] = va; }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // Threads: 256.  GT = query heads per CTA (all sharing one kv head),
 // R = sub-rows of 16 rows per q-block.
 template <int D, int GT, int R>
@@ -251,23 +275,34 @@ __global__ void __launch_bounds__(256, 2) kap_score_select_kernel(ScoreArgs a) {
   const int8_t* kq = a.kq + (static_cast<long>(kv) * a.nqb_total + qb0) * D;
   const float* ksp = a.ks + static_cast<long>(kv) * a.nqb_total + qb0;
   const int ntiles = (n + 7) >> 3;
-  for (int tile = warp; tile < ntiles; tile += 8) {
-    const int key = tile * 8 + gq;
-    uint32_t bfr[QR];
-    if (key < n) {
+  // key fragments and scales of a tile of 8 keys (zeros past n); fetched one tile ahead
+  auto load_tile = [&](int tl, uint32_t (&bf)[QR], float& s0, float& s1) {
+    const int key = tl * 8 + gq;
+    if (tl < ntiles && key < n) {
       const uint32_t* src = reinterpret_cast<const uint32_t*>(kq + static_cast<long>(key) * D + qd * QB);
 #pragma unroll
       for (int x = 0; x < QR; x += 4) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + x));
-        bfr[x] = v.x; bfr[x + 1] = v.y; bfr[x + 2] = v.z; bfr[x + 3] = v.w;
+        bf[x] = v.x; bf[x + 1] = v.y; bf[x + 2] = v.z; bf[x + 3] = v.w;
       }
     } else {
 #pragma unroll
-      for (int x = 0; x < QR; ++x) bfr[x] = 0u;
+      for (int x = 0; x < QR; ++x) bf[x] = 0u;
     }
+    const int k0 = tl * 8 + 2 * qd;
+    s0 = (tl < ntiles && k0 < n) ? __ldg(ksp + k0) : 0.0f;
+    s1 = (tl < ntiles && k0 + 1 < n) ? __ldg(ksp + k0 + 1) : 0.0f;
+  };
+  uint32_t bnext[QR];
+  float ks0n, ks1n;
+  load_tile(warp, bnext, ks0n, ks1n);
+  for (int tile = warp; tile < ntiles; tile += 8) {
+    uint32_t bfr[QR];
+#pragma unroll
+    for (int x = 0; x < QR; ++x) bfr[x] = bnext[x];
+    const float ks0 = ks0n, ks1 = ks1n;
+    load_tile(tile + 8, bnext, ks0n, ks1n);
     const int key0 = tile * 8 + 2 * qd;
-    const float ks0 = (key0 < n) ? __ldg(ksp + key0) : 0.0f;
-    const float ks1 = (key0 + 1 < n) ? __ldg(ksp + key0 + 1) : 0.0f;
 #pragma unroll
     for (int mt = 0; mt < GT; ++mt) {
       int c[4] = {0, 0, 0, 0};
@@ -327,30 +362,105 @@ __global__ void __launch_bounds__(256, 2) kap_score_select_kernel(ScoreArgs a) {
   }
   __syncthreads();
 
-  // ---- phase 4: bitonic sort of each head's npow2 keys (ascending)
-  const int half = GT * npow2 / 2;
-  for (int k = 2; k <= npow2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int idx = tid; idx < half; idx += 256) {
-        const int seg = idx / (npow2 / 2);
-        const int li = idx % (npow2 / 2);
-        const int x = (li / jj) * 2 * jj + (li % jj);
-        uint64_t* base = keys + seg * a.npow2_max;
-        const uint64_t va = base[x], vb = base[x + jj];
-        const bool asc = (x & k) == 0;
-        if ((va > vb) == asc) { base[x] = vb; base[x + jj] = va; }
+  // ---- phase 4: each head's k_i smallest keys, in ascending order
+  // The 64-bit keys are unique (they end in the block index), so a radix
+  // select from the top byte down finds exactly the k_i smallest: at every
+  // pass the bucket holding the k-th key is narrowed until all of it is
+  // kept.  Only those keys are then sorted.  When every candidate is kept
+  // (k_i = n), or the small buffers do not fit, all candidates are sorted.
+  const int k_i = static_cast<int>(max(1LL, (static_cast<long long>(n) * a.bp + 9999) / 10000));
+  int kpow = 1;
+  while (kpow < k_i) kpow <<= 1;
+  const bool select_path = (k_i < n) && (GT * 256 * 4 + GT * kpow * 8 <= R * COLS * 4);
+  const uint64_t* out_keys = keys;
+  int out_stride = a.npow2_max;
+  if (select_path) {
+    int* hist = reinterpret_cast<int*>(subsum);                               // [GT][256]
+    uint64_t* sel = reinterpret_cast<uint64_t*>(hist + GT * 256);             // [GT][kpow]
+    unsigned long long* st_prefix = reinterpret_cast<unsigned long long*>(red_s);
+    unsigned long long* st_mask = st_prefix + GT;
+    int* st_need = reinterpret_cast<int*>(st_mask + GT);
+    int* st_done = st_need + GT;
+    int* st_cnt = st_done + GT;
+    if (tid < GT) {
+      st_prefix[tid] = 0ull;
+      st_mask[tid] = 0ull;
+      st_need[tid] = k_i;
+      st_done[tid] = 0;
+      st_cnt[tid] = 0;
+    }
+    __syncthreads();
+    for (int pass = 0; pass < 8; ++pass) {
+      const int shift = 56 - 8 * pass;
+      for (int x = tid; x < GT * 256; x += 256) hist[x] = 0;
+      __syncthreads();
+      for (int mt = 0; mt < GT; ++mt) {
+        if (st_done[mt]) continue;
+        const unsigned long long pm = st_mask[mt], pv = st_prefix[mt];
+        for (int j = tid; j < n; j += 256) {
+          const uint64_t key = keys[mt * a.npow2_max + j];
+          if ((key & pm) == pv) atomicAdd(&hist[mt * 256 + static_cast<int>((key >> shift) & 255u)], 1);
+        }
       }
       __syncthreads();
+      if (warp < GT && !st_done[warp]) {
+        int c[8];
+        int sum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c[e] = hist[warp * 256 + 8 * lane + e];
+          sum += c[e];
+        }
+        int inc = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, inc, off);
+          if (lane >= off) inc += y;
+        }
+        const int need = st_need[warp];
+        const int excl = inc - sum;
+        if (excl < need && need <= inc) {   // this lane's bins hold the need-th key
+          int below = excl, e = 0;
+          while (below + c[e] < need) below += c[e++];
+          const int rest = need - below;
+          st_need[warp] = rest;
+          st_prefix[warp] |= static_cast<unsigned long long>(8 * lane + e) << shift;
+          st_mask[warp] |= 255ull << shift;
+          st_done[warp] = (c[e] == rest) ? 1 : 0;
+        }
+      }
+      __syncthreads();
+      int all = 1;
+      for (int mt = 0; mt < GT; ++mt) all &= st_done[mt];
+      if (all) break;
     }
+    for (int x = tid; x < GT * kpow; x += 256) sel[x] = ~0ull;
+    __syncthreads();
+    for (int mt = 0; mt < GT; ++mt) {
+      const unsigned long long pm = st_mask[mt], pv = st_prefix[mt];
+      for (int j = tid; j < n; j += 256) {
+        const uint64_t key = keys[mt * a.npow2_max + j];
+        if ((key & pm) <= pv) {
+          const int pos = atomicAdd(&st_cnt[mt], 1);
+          if (pos < kpow) sel[mt * kpow + pos] = key;
+          else report(a.status, kErrBounds, 0x201);
+        }
+      }
+    }
+    __syncthreads();
+    bitonic_sort(sel, GT, kpow, kpow);
+    out_keys = sel;
+    out_stride = kpow;
+  } else {
+    bitonic_sort(keys, GT, npow2, a.npow2_max);
   }
 
   // ---- phase 5: emit the first k_i entries
-  const int k_i = static_cast<int>(max(1LL, (static_cast<long long>(n) * a.bp + 9999) / 10000));
   for (int x = tid; x < GT * a.kmax; x += 256) {
     const int mt = x / a.kmax, t = x % a.kmax;
     const long o = (static_cast<long>(h0 + mt) * a.nqb_total + I) * a.kmax + t;
     if (t < k_i) {
-      const uint64_t key = keys[mt * a.npow2_max + t];
+      const uint64_t key = out_keys[mt * out_stride + t];
       a.order[o] = static_cast<int32_t>(key & 0x7FFFFFFFu);
       a.hrm[o] = static_cast<uint8_t>((key >> 63) ? 0 : 1);
     } else {
@@ -360,7 +470,7 @@ __global__ void __launch_bounds__(256, 2) kap_score_select_kernel(ScoreArgs a) {
   }
   if (tid < GT) {
     int c = 0;
-    while (c < k_i && !(keys[tid * a.npow2_max + c] >> 63)) ++c;
+    while (c < k_i && !(out_keys[tid * out_stride + c] >> 63)) ++c;
     const long o = static_cast<long>(h0 + tid) * a.nqb_total + I;
     a.count[o] = k_i;
     a.n_hrm[o] = c;
