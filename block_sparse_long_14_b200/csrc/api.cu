@@ -63,8 +63,10 @@ int check_shape(const cosa_shape_t* s) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Workspace: status block, pooled int8 keys [Hkv, NQB, d], key scales
+// [Hkv, NQB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d].
 struct WsLayout {
-  size_t kq_off, ks_off, total;
+  size_t kq_off, ks_off, qa_off, total;
 };
 
 WsLayout ws_layout(const cosa_shape_t& s) {
@@ -72,8 +74,27 @@ WsLayout ws_layout(const cosa_shape_t& s) {
   w.kq_off = kStatusBytes;
   const size_t kq_bytes = static_cast<size_t>(s.num_kv_heads) * s.total_qblocks * s.head_dim;
   w.ks_off = align_up(w.kq_off + kq_bytes, 256);
-  w.total = align_up(w.ks_off + static_cast<size_t>(s.num_kv_heads) * s.total_qblocks * 4, 256);
+  w.qa_off = align_up(w.ks_off + static_cast<size_t>(s.num_kv_heads) * s.total_qblocks * 4, 256);
+  const size_t qa_bytes =
+      static_cast<size_t>(s.num_q_heads) * s.total_qblocks * (s.block_size / 16 + 1) * s.head_dim;
+  w.total = align_up(w.qa_off + qa_bytes, 256);
   return w;
+}
+
+// Radix-select scratch of the select kernel: histograms plus a buffer for the
+// kept keys (rounded up to a power of two), shrunk if shared memory is short;
+// rows whose keys do not fit fall back to a full in-place sort.
+int select_scratch_bytes(const cosa_shape_t& s, int kmax, int GT, int npow2_max) {
+  int kpow = 8;   // room for all HRM keys of a row (at most b / 16 <= 8) before the cut at k_i
+  while (kpow < kmax) kpow <<= 1;
+  if (kpow > npow2_max) kpow = npow2_max;
+  int bytes = GT * 256 * 4 + GT * kpow * 8;
+  while (kpow > 1 && (select_smem_bytes(s.head_dim, GT, npow2_max, bytes) > 200 * 1024 ||
+                      select_tc_smem_bytes(GT, npow2_max, bytes) > 220 * 1024)) {
+    kpow >>= 1;
+    bytes = GT * 256 * 4 + GT * kpow * 8;
+  }
+  return bytes;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
@@ -93,14 +114,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle and 64-element (128-byte) inner boxes.
+// Tensor map with 128-byte swizzle and 128-byte inner boxes (bf16 unless stated).
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
-              const cuuint32_t* box) {
+              const cuuint32_t* box, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint32_t elem[3] = {1, 1, 1};
   std::memset(m, 0, sizeof(*m));
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
+  return fn(m, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
             strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -200,7 +221,21 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   sa.kmax = kmax;
   sa.bp = bp;
   sa.npow2_max = next_pow2(ceil_div(shape->max_seqlen, shape->block_size));
-  if (launch_score(sa, proxy_group(*shape), st) != cudaSuccess) return COSA_ERR_CUDA;
+  sa.qa = reinterpret_cast<int8_t*>(ws + w.qa_off);
+  const int GT = proxy_group(*shape);
+  sa.scratch_bytes = select_scratch_bytes(*shape, kmax, GT, sa.npow2_max);
+  if (launch_qpool(sa, GT, st) != cudaSuccess) return COSA_ERR_CUDA;
+  if (shape->head_dim == 128) {
+    // int8 key vectors as a [Hkv * NQB, 128] byte matrix for the tcgen05 score tiles
+    CUtensorMap kq_map;
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(shape->num_kv_heads) * shape->total_qblocks};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, 128};
+    if (!make_map(&kq_map, sa.kq, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return COSA_ERR_CUDA;
+    if (launch_select_tc(sa, GT, kq_map, st) != cudaSuccess) return COSA_ERR_CUDA;
+  } else {
+    if (launch_select(sa, GT, st) != cudaSuccess) return COSA_ERR_CUDA;
+  }
   return COSA_OK;
 }
 

@@ -35,7 +35,9 @@ struct ScoreArgs {
   int32_t* n_hrm;
   uint8_t* hrm;
   Status* status;
+  int8_t* qa;          // pooled int8 query vectors [Hq, NQB, R + 1, d] (two-stage path only)
   int batch, num_q_heads, num_kv_heads, head_dim, block_size, nqb_total, kmax, bp, npow2_max;
+  int scratch_bytes;   // radix-select scratch of the select kernel
 };
 
 struct RemapArgs {
@@ -70,8 +72,14 @@ struct OskArgs {
 };
 
 size_t score_smem_bytes(int D, int GT, int R, int npow2_max);
+size_t select_smem_bytes(int D, int GT, int npow2_max, int scratch_bytes);
 cudaError_t launch_kpool(const KPoolArgs& a, cudaStream_t stream);
-cudaError_t launch_score(const ScoreArgs& a, int GT, cudaStream_t stream);
+cudaError_t launch_score(const ScoreArgs& a, int GT, cudaStream_t stream);    // fused pool + select
+cudaError_t launch_qpool(const ScoreArgs& a, int GT, cudaStream_t stream);    // pool -> a.qa
+cudaError_t launch_select(const ScoreArgs& a, int GT, cudaStream_t stream);   // a.qa -> lists
+// a.qa -> lists on tcgen05 int8 MMAs (head_dim 128); kq_map covers a.kq as [Hkv * NQB, 128] int8
+cudaError_t launch_select_tc(const ScoreArgs& a, int GT, const CUtensorMap& kq_map, cudaStream_t stream);
+size_t select_tc_smem_bytes(int GT, int npow2_max, int scratch_bytes);
 cudaError_t launch_remap(const RemapArgs& a, cudaStream_t stream);
 cudaError_t launch_osk(const OskArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                        const CUtensorMap& vmap, int head_dim, cudaStream_t stream);
