@@ -26,9 +26,11 @@
 //              its own half of the S columns in TMEM, partial row sums, lazy
 //              rescaling of its half of O in TMEM, the epilogue O / l.
 //   warp 8     producer: page remap (order -> page_table) and TMA loads of the
-//              Q tile and of each block's K and V pages into 3-stage rings; a
-//              block ending past the sequence is copied by hand with zero
-//              fill so no stray page slot reaches an MMA.
+//              Q tile and of each block's K and V pages into 3-stage rings.
+//              Block and page ids are loaded two blocks ahead of the copies and
+//              lane u issues the boxes of page u; a block ending past the
+//              sequence is copied by hand with zero fill so no stray page slot
+//              reaches an MMA.
 //   warp 9     MMA issuer: S = Q K^T (M=128, N=b, K=d; both operands in shared
 //              memory) into one of two TMEM S buffers, then O += P V
 //              (M=128, N=d, K=b) with P read from TMEM, unless the tile voted
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t* ord = a.order + row_id * a.kmax;
   const int32_t* pt_row = a.page_table + static_cast<long>(s) * a.max_pages_per_seq;
 
-  if (tid == 0) {
+  if (tid == kProducerWarp * 32) {
     mbar_init(&bars->q_full, 1);
     for (int x = 0; x < kStages; ++x) {
       mbar_init(&bars->k_full[x], 1);
@@ -195,6 +197,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->mma_drain, 1);
     bars->abort = 0;
     mbar_fence_init();
+    if (n > 0) {
+      prefetch_tmap(&qmap);
+      prefetch_tmap(&kmap);
+      prefetch_tmap(&vmap);
+      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * (kBQ * 128), &qmap, &bars->q_full, c * 64, h, tok0 + i * b);
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
@@ -218,47 +228,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k_armed[kStages], v_armed[kStages];
     for (int x = 0; x < kStages; ++x) k_armed[x] = v_armed[x] = -1;
     bool ok = true;
-    if (lane == 0) {
-      prefetch_tmap(&qmap);
-      prefetch_tmap(&kmap);
-      prefetch_tmap(&vmap);
-      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * (kBQ * 128), &qmap, &bars->q_full, c * 64, h, tok0 + i * b);
-    }
     const int ppb = b / a.page_size;
+    // Lane u < ppb holds page u of a block.  The loads run ahead of the
+    // copies: the id of block t+2 and the page ids of block t+1 are already
+    // in registers when block t is issued, so the order -> page table chain
+    // of dependent loads never stalls a copy.
+    auto block_id = [&](int t) { return t < n ? __ldg(ord + t) : -1; };
+    auto page_of = [&](int jb) {
+      return (lane < ppb && jb >= 0 && jb < nkb && jb * b + lane * a.page_size < L) ? __ldg(pt_row + jb * ppb + lane)
+                                                                                     : -1;
+    };
+    int j_c = block_id(0);
+    int pg_c = page_of(j_c);
+    int j_n = block_id(1);
+    int pg_n = page_of(j_n);
+    int j_nn = block_id(2);
     for (int t = 0; t < n && ok; ++t) {
       const int slot = t % kStages, use = t / kStages;
-      int j = __ldg(ord + t);
+      int j = j_c;
+      const int page = pg_c;
       bool jvalid = (j >= 0 && j < nkb);
       if (!jvalid) {
         if (lane == 0) report(a.status, kErrBounds, 0x302);
         j = 0;
       }
       const int nvalid = jvalid ? min(b, L - j * b) : 0;
-      // Page ids of the block (lane u holds page u); a bad id sends the block down the checked path.
-      int page = -1;
-      if (lane < ppb && jvalid && j * b + lane * a.page_size < L) page = __ldg(pt_row + j * ppb + lane);
+      // a bad page id sends the block down the checked path
       const bool pages_ok = __all_sync(0xffffffffu, lane >= ppb || (page >= 0 && page < a.num_pages));
       const bool via_tma = jvalid && nvalid == b && pages_ok;
+      const int row = (page * a.num_kv_heads + g) * a.page_size;  // lane u < ppb: first pool row of page u
+      // look-ahead loads, consumed one and two blocks later
+      const int pg_nn = page_of(j_nn);
+      const int j_nnn = block_id(t + 3);
       for (int kvsel = 0; kvsel < 2 && ok; ++kvsel) {
         uint64_t* full = kvsel == 0 ? &bars->k_full[slot] : &bars->v_full[slot];
         uint64_t* empty = kvsel == 0 ? &bars->k_empty[slot] : &bars->v_empty[slot];
         unsigned char* stage = (kvsel == 0 ? sK : sV) + slot * C::KV_BYTES;
         const CUtensorMap* map = kvsel == 0 ? &kmap : &vmap;
-        if (use >= 1 && lane == 0) ok = mbar_wait(empty, (use - 1) & 1, a.wait_limit, abort, a.status, 0x10 + kvsel);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (use >= 1) ok = mbar_wait(empty, (use - 1) & 1, a.wait_limit, abort, a.status, 0x10 + kvsel);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (via_tma) {
           if (lane == 0) mbar_arrive_expect_tx(full, C::KV_BYTES);
-          for (int u = 0; u < ppb; ++u) {
-            const int pg = __shfl_sync(0xffffffffu, page, u);
-            if (lane == 0) {
-              const int row = (pg * a.num_kv_heads + g) * a.page_size;
+          __syncwarp();
+          if (lane < ppb) {
 #pragma unroll
-              for (int c = 0; c < D / 64; ++c)
-                tma_load_2d(stage + c * (BK * 128) + u * a.page_size * 128, map, full, c * 64, row);
-            }
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_2d(stage + c * (BK * 128) + lane * a.page_size * 128, map, full, c * 64, row);
           }
           __syncwarp();
         } else {
@@ -267,6 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (kvsel == 0) k_armed[slot] = use; else v_armed[slot] = use;
       }
+      j_c = j_n;
+      pg_c = pg_n;
+      j_n = j_nn;
+      pg_n = pg_nn;
+      j_nn = j_nnn;
     }
     // drain: every load this warp started has landed before the CTA exits
     if (lane == 0) {
