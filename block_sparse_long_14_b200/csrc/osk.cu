@@ -32,12 +32,13 @@
 //              sequence is copied by hand with zero fill so no stray page slot
 //              reaches an MMA.
 //   warp 9     MMA issuer: S = Q K^T (M=128, N=b, K=d; both operands in shared
-//              memory) into one of two TMEM S buffers, then O += P V
-//              (M=128, N=d, K=b) with P read from TMEM, unless the tile voted
-//              to skip; completion is signalled with tcgen05.commit.
+//              memory) into one of three TMEM S buffers (block t uses t % 3),
+//              then O += P V (M=128, N=d, K=b) with P read from TMEM, unless
+//              the tile voted to skip; completion is signalled with
+//              tcgen05.commit.  S of block t+2 is issued right after P V of
+//              block t, a whole block ahead of the softmax warps.
 // The tensor pipe executes one thread's MMAs in issue order, so P V of block
-// t-2 has read its P before S of block t overwrites the same columns; S for
-// block t+1 is computed while the softmax warps work on block t.
+// t-1 has read its P before S of block t+2 overwrites the same columns.
 // Every wait is bounded; on expiry the CTA records COSA_ERR_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
 #include <cstdint>
@@ -64,7 +65,7 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2];
+  uint64_t s_full[3];
   uint64_t p_full[2];   // softmax verdict (and P, if kept) for block t, by t & 1
   uint64_t o_done[2];   // P V of kept block c has completed, by c & 1
   uint64_t mma_drain;
@@ -87,10 +88,10 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_V + kStages * KV_BYTES;
   static constexpr int HALF = BK / 2;   // key columns per softmax thread
   static constexpr int KPH = HALF / 16; // K=16 MMA steps per half
-  static constexpr int TMEM_S0 = 0;
-  static constexpr int TMEM_S1 = BK;
-  static constexpr int TMEM_O = 2 * BK;
-  static constexpr int TMEM_NEED = 2 * BK + D;
+  // three S buffers (block t uses t % 3), so S of block t+2 can be issued
+  // right after P V of block t, while P of block t+1 still occupies its own
+  static constexpr int TMEM_O = 3 * BK;
+  static constexpr int TMEM_NEED = 3 * BK + D;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                    : TMEM_NEED <= 256 ? 256 : 512;
   // Shared memory is padded so that the CTAs resident on one SM never ask
@@ -189,8 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_full[x], 1);
       mbar_init(&bars->v_empty[x], 1);
     }
+    for (int x = 0; x < 3; ++x) mbar_init(&bars->s_full[x], 1);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&bars->s_full[x], 1);
       mbar_init(&bars->p_full[x], kSoftmaxThreads);
       mbar_init(&bars->o_done[x], 1);
     }
@@ -303,47 +304,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
       bool ok = mbar_wait(&bars->q_full, 0, a.wait_limit, abort, a.status, 0x20);
       int kept = 0;
-      for (int t = 0; t <= n && ok; ++t) {
-        if (t < n) {
-          const int slot = t % kStages, use = t / kStages;
-          ok = mbar_wait(&bars->k_full[slot], use & 1, a.wait_limit, abort, a.status, 0x21);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t d_s = tmem + ((t & 1) ? C::TMEM_S1 : C::TMEM_S0);
+      // S = Q K^T of block t into S buffer t % 3
+      auto issue_s = [&](int t) -> bool {
+        const int slot = t % kStages, use = t / kStages;
+        if (!mbar_wait(&bars->k_full[slot], use & 1, a.wait_limit, abort, a.status, 0x21)) return false;
+        tc_fence_after();
+        const uint32_t d_s = tmem + (t % 3) * BK;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ad = sw128_desc(q_base + (ks >> 2) * (kBQ * 128) + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(k_base + slot * C::KV_BYTES + (ks >> 2) * (BK * 128) + (ks & 3) * 32, 16, 1024);
-            tc_mma_ss(d_s, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
-          }
-          tc_commit(&bars->s_full[t & 1]);
-          tc_commit(&bars->k_empty[slot]);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ad = sw128_desc(q_base + (ks >> 2) * (kBQ * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(k_base + slot * C::KV_BYTES + (ks >> 2) * (BK * 128) + (ks & 3) * 32, 16, 1024);
+          tc_mma_ss(d_s, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
         }
-        if (t >= 1) {
-          const int u = t - 1, vslot = u % kStages, vuse = u / kStages;
-          ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, a.wait_limit, abort, a.status, 0x23);
-          if (ok) ok = mbar_wait(&bars->v_full[vslot], vuse & 1, a.wait_limit, abort, a.status, 0x24);
-          if (!ok) break;
-          tc_fence_after();
-          const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[u & 1]);
-          if (!skip) {
-            const uint32_t p_tmem = tmem + ((u & 1) ? C::TMEM_S1 : C::TMEM_S0);
-            const uint32_t d_o = tmem + C::TMEM_O;
+        tc_commit(&bars->s_full[t % 3]);
+        tc_commit(&bars->k_empty[slot]);
+        return true;
+      };
+      if (ok && n > 0) ok = issue_s(0);
+      if (ok && n > 1) ok = issue_s(1);
+      for (int u = 0; u < n && ok; ++u) {
+        const int vslot = u % kStages, vuse = u / kStages;
+        ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, a.wait_limit, abort, a.status, 0x23);
+        if (ok) ok = mbar_wait(&bars->v_full[vslot], vuse & 1, a.wait_limit, abort, a.status, 0x24);
+        if (!ok) break;
+        tc_fence_after();
+        const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[u & 1]);
+        if (!skip) {
+          const uint32_t p_tmem = tmem + (u % 3) * BK;
+          const uint32_t d_o = tmem + C::TMEM_O;
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              // P of keys [16kk, 16kk+16): half kk / KPH wrote its P into the first
-              // HALF/2 columns of its own S half
-              const uint32_t a_t = p_tmem + (kk / C::KPH) * C::HALF + (kk % C::KPH) * 8;
-              const uint64_t bd = sw128_desc(v_base + vslot * C::KV_BYTES + kk * 2048, BK * 128, 1024);
-              tc_mma_ts(d_o, a_t, bd, C::IDESC_PV, (kept > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc_commit(&bars->v_empty[vslot]);
-            tc_commit(&bars->o_done[kept & 1]);
-            ++kept;
-          } else {
-            mbar_arrive(&bars->v_empty[vslot]);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // P of keys [16kk, 16kk+16): half kk / KPH wrote its P into the first
+            // HALF/2 columns of its own S half
+            const uint32_t a_t = p_tmem + (kk / C::KPH) * C::HALF + (kk % C::KPH) * 8;
+            const uint64_t bd = sw128_desc(v_base + vslot * C::KV_BYTES + kk * 2048, BK * 128, 1024);
+            tc_mma_ts(d_o, a_t, bd, C::IDESC_PV, (kept > 0 || kk > 0) ? 1u : 0u);
           }
+          tc_commit(&bars->v_empty[vslot]);
+          tc_commit(&bars->o_done[kept & 1]);
+          ++kept;
+        } else {
+          mbar_arrive(&bars->v_empty[vslot]);
         }
+        // S of block u+2 reuses the buffer of block u-1, whose P V was issued above
+        if (u + 2 < n) ok = issue_s(u + 2);
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
       tc_commit(&bars->mma_drain);
@@ -364,10 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int j_next = __ldg(ord);
     for (int t = 0; t < n; ++t) {
       const int sb = t & 1;
-      const uint32_t s_cols = lane_base + (sb ? C::TMEM_S1 : C::TMEM_S0) + col0;
+      const int sbuf = t % 3;
+      const uint32_t s_cols = lane_base + sbuf * BK + col0;
       const int j = j_next;
       if (t + 1 < n) j_next = __ldg(ord + t + 1);
-      bool ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, a.wait_limit, abort, a.status, 0x30);
+      bool ok = mbar_wait(&bars->s_full[sbuf], (t / 3) & 1, a.wait_limit, abort, a.status, 0x30);
       ok = __all_sync(0xffffffffu, ok) && !aborted;
       float sv[C::HALF];
       if (ok) {
