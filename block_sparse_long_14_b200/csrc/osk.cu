@@ -435,18 +435,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = __any_sync(0xffffffffu, need);
         if (rescale && row_valid) new_ref = m_new;
       }
-      // P = exp2(s * log2e/sqrt(d) - ref) in bf16; partial row sum of the rounded values
+      // P = exp2(s * log2e/sqrt(d) - ref) in bf16; partial row sum of the fp32 values.
+      // Rows past the sequence end need no masking here: a row of P only feeds the
+      // same row of O, and those rows of O are never written out.
       uint32_t pk[C::HALF / 2];
-      float ls0 = 0.0f, ls1 = 0.0f;
+      float2 ls = make_float2(0.0f, 0.0f);
       const float nb = (new_ref == -INFINITY) ? 0.0f : -new_ref;
+      const float2 sl2x2 = make_float2(sl2, sl2), nbx2 = make_float2(nb, nb);
 #pragma unroll
       for (int e = 0; e < C::HALF / 2; ++e) {
-        const float p0 = ex2_approx(fmaf(sv[2 * e], sl2, nb));
-        const float p1 = ex2_approx(fmaf(sv[2 * e + 1], sl2, nb));
-        pk[e] = row_valid ? pack_bf16x2(p0, p1) : 0u;
-        ls0 += __uint_as_float(pk[e] << 16);
-        ls1 += __uint_as_float(pk[e] & 0xFFFF0000u);
+        // two logits per packed fp32 FMA, two sums per packed add
+        const float2 x = fma_f32x2(make_float2(sv[2 * e], sv[2 * e + 1]), sl2x2, nbx2);
+        const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        pk[e] = pack_bf16x2(pv.x, pv.y);
+        ls = add_f32x2(ls, pv);
       }
+      const float ls0 = ls.x, ls1 = ls.y;
       if (rescale) {
         // O must be complete up to the last kept block before it is re-based
         bool okw = mbar_wait(&bars->o_done[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status,
