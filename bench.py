@@ -48,6 +48,25 @@ def peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def measured_traffic():
+    """DRAM bytes per OSK launch from the committed ncu launch list, or None
+    when the kernel's sources changed since those counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "osk_traffic_llama8b_128k.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    h = hashlib.sha256()
+    for f in d["source_files"]:
+        fp = os.path.join(ROOT, f)
+        if not os.path.exists(fp):
+            return None
+        h.update(open(fp, "rb").read())
+    if h.hexdigest() != d["source_sha256"]:
+        return None
+    return d["dram_read_bytes_per_launch"] + d["dram_write_bytes_per_launch"]
+
+
 def rank_seed(cfg, rank, world):
     """Each rank prefills its own independent layer: distinct seeds for N > 1,
     the workload's own seed at N = 1."""
@@ -410,15 +429,16 @@ def run_cosa(args, rank, world, local_rank):
         "realized_budget": {"stage1": visited / nqb_rows, "stage2": (visited - skipped) / nqb_rows,
                             "skip_ratio": skipped / visited},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": attn_tflops / pk["bf16_sustained"], "traffic": None,
+                     "frac": attn_tflops / pk["bf16_sustained"],
+                     "traffic": measured_traffic() if CONFIG_ID == args.config else None,
                      "kernel": "osk_kernel<128,128>",
                      "peak_source": f"{pk['source']} bf16_tflops_sustained (kernel timed inside repeated steps)",
                      "algorithmic": f"{exec_flops:.4e} FLOP per launch = 2*128*128*128 * (visited + kept)"},
         "proxy_roofline": {"bound": "hbm", "achieved": proxy_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                            "frac": proxy_gbs / pk["hbm_gbs"], "algorithmic_bytes": proxy_bytes,
-                           "kernels": "kpool + kap_score_select"},
+                           "kernels": "kpool + qpool + kap_select_tc"},
         "clocks": clocks,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,   # kpool, qpool, select, osk per step
         "e2e": e2e,
         **extra,
     }
