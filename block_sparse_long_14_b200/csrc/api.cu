@@ -230,7 +230,7 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
     CUtensorMap kq_map;
     const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(shape->num_kv_heads) * shape->total_qblocks};
     const cuuint64_t strides[1] = {128};
-    const cuuint32_t box[2] = {128, 128};
+    const cuuint32_t box[2] = {128, 64};   // 64 key blocks x 128 int8 dims per score tile
     if (!make_map(&kq_map, sa.kq, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return COSA_ERR_CUDA;
     if (launch_select_tc(sa, GT, kq_map, st) != cudaSuccess) return COSA_ERR_CUDA;
   } else {

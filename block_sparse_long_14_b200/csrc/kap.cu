@@ -606,24 +606,21 @@ __device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-// 16 TMEM lanes x 64 columns: thread t receives lane t/4 in registers
+// 16 TMEM lanes x 32 columns: thread t receives lane t/4 in registers
 // 4c, 4c+1 and lane t/4 + 8 in registers 4c+2, 4c+3, at columns
-// 8c + 2 (t % 4) + {0, 1}, c = 0..7.
-__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t* r) {
+// 8c + 2 (t % 4) + {0, 1}, c = 0..3.
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t* r) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
-        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
-        "=r"(r[30]), "=r"(r[31])
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
 
-constexpr int kTcN = 128;                 // candidate key blocks per score tile
-constexpr int kTcRing = 2;                // key tiles in flight (shared memory caps CTAs per SM)
+constexpr int kTcN = 64;                  // candidate key blocks per score tile
+constexpr int kTcRing = 2;                // key tiles in flight
+constexpr int kTcTmemCols = 2 * kTcN;     // two accumulators: 3 CTAs per SM fit in TMEM
 constexpr uint32_t kTcWaitLimit = 1u << 22;
 
 // Instruction descriptor of kind::i8: D format S32 (2) at bit 4, A and B
@@ -645,11 +642,13 @@ size_t select_tc_smem_bytes(int GT, int npow2_max, int scratch_bytes) {
 // M = 64 rows: head mt's vectors occupy rows 16 mt .. 16 mt + R, which
 // tcgen05 places in TMEM lanes 32 mt .. 32 mt + R of quadrant mt, so warp w
 // (quadrant w % 4, key columns half w / 4) reads exactly its head's scores
-// with the 16-lane TMEM load.  N = 128 key blocks per MMA, K = 128 dims in
+// with the 16-lane TMEM load.  N = 64 key blocks per MMA, K = 128 dims in
 // 4 steps of 32; the int8 key tiles arrive by TMA (128B swizzle), two tiles
-// in flight, two TMEM accumulators (256 columns).
+// in flight, two TMEM accumulators (128 columns).  The small tiles keep the
+// shared memory and TMEM of a CTA low enough for three CTAs per SM: the
+// kernel is latency-bound, so resident CTAs are what hides the latency.
 template <int GT, int R>
-__global__ void __launch_bounds__(256, 2) kap_select_tc_kernel(const __grid_constant__ CUtensorMap kq_map, ScoreArgs a) {
+__global__ void __launch_bounds__(256, 3) kap_select_tc_kernel(const __grid_constant__ CUtensorMap kq_map, ScoreArgs a) {
   constexpr int D = 128;
   constexpr uint32_t IDESC = idesc_s8_s32(64, kTcN);
   extern __shared__ __align__(1024) unsigned char smem_tc[];
@@ -684,8 +683,24 @@ __global__ void __launch_bounds__(256, 2) kap_select_tc_kernel(const __grid_cons
     mbar_fence_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kTcTmemCols);
     tmem_relinquish();
+  }
+  const int ntiles = (n + kTcN - 1) / kTcN;
+  const int row0 = tl.kv * a.nqb_total + tl.qb0;   // Kq row of key block 0 of this sequence
+  // key tiles cycle through a ring of kTcRing shared-memory slots (b_full[slot]);
+  // accumulators alternate between two TMEM buffers (mma_done[t & 1])
+  uint64_t* b_full = bars;
+  uint64_t* mma_done = bars + kTcRing;
+  auto issue_load = [&](int t) {
+    const int slot = t % kTcRing;
+    mbar_arrive_expect_tx(&b_full[slot], kTcN * 128);
+    tma_load_2d(sB + slot * (kTcN * 128), &kq_map, &b_full[slot], 0, row0 + t * kTcN);
+  };
+  // the first key tiles are requested before the query vectors are staged
+  if (tid == 0) {
+    prefetch_tmap(&kq_map);
+    for (int t = 0; t < kTcRing && t < ntiles; ++t) issue_load(t);
   }
   // A operand: rows 16 mt + v (v <= R) = head mt's vector v; other rows zero.  128B-swizzled K-major.
   for (int x = tid; x < 64 * 8; x += 256) {
@@ -707,18 +722,7 @@ __global__ void __launch_bounds__(256, 2) kap_select_tc_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int ntiles = (n + kTcN - 1) / kTcN;
-  const int row0 = tl.kv * a.nqb_total + tl.qb0;   // Kq row of key block 0 of this sequence
   const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
-  // key tiles cycle through a ring of kTcRing shared-memory slots (b_full[slot]);
-  // accumulators alternate between two TMEM buffers (mma_done[t & 1])
-  uint64_t* b_full = bars;
-  uint64_t* mma_done = bars + kTcRing;
-  auto issue_load = [&](int t) {
-    const int slot = t % kTcRing;
-    mbar_arrive_expect_tx(&b_full[slot], kTcN * 128);
-    tma_load_2d(sB + slot * (kTcN * 128), &kq_map, &b_full[slot], 0, row0 + t * kTcN);
-  };
   auto issue_mma = [&](int t) {
     const int slot = t % kTcRing;
     if (!mbar_wait(&b_full[slot], (t / kTcRing) & 1, kTcWaitLimit, abort_flag, a.status, 0x210)) return;
@@ -731,11 +735,7 @@ __global__ void __launch_bounds__(256, 2) kap_select_tc_kernel(const __grid_cons
     }
     tc_commit(&mma_done[t & 1]);
   };
-  if (tid == 0) {
-    prefetch_tmap(&kq_map);
-    for (int t = 0; t < kTcRing && t < ntiles; ++t) issue_load(t);
-    issue_mma(0);
-  }
+  if (tid == 0) issue_mma(0);
 
   const int q = warp & 3, half = warp >> 2, v = lane >> 2;
   float best_s[2] = {-FLT_MAX, -FLT_MAX};
@@ -747,14 +747,14 @@ __global__ void __launch_bounds__(256, 2) kap_select_tc_kernel(const __grid_cons
     // the MMA of tile t has read its key slot: refill it right away
     if (tid == 0 && ok && t + kTcRing < ntiles) issue_load(t + kTcRing);
     if (q < GT && __all_sync(0xffffffffu, ok)) {
-      uint32_t r[32];
-      tmem_ld_16x256b_x8(tmem + (static_cast<uint32_t>(32 * q) << 16) + (t & 1) * kTcN + half * 64, r);
+      uint32_t r[16];
+      tmem_ld_16x256b_x4(tmem + (static_cast<uint32_t>(32 * q) << 16) + (t & 1) * kTcN + half * (kTcN / 2), r);
       tc_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int j = t * kTcN + half * 64 + 8 * c + 2 * (lane & 3) + e;
+          const int j = t * kTcN + half * (kTcN / 2) + 8 * c + 2 * (lane & 3) + e;
           if (j < n) {
             const float ks = sKs[j];
             const float s_lo = __fmul_rn(static_cast<float>(static_cast<int>(r[4 * c + e])), ks);
@@ -801,7 +801,7 @@ __global__ void __launch_bounds__(256, 2) kap_select_tc_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, kTcTmemCols);
   select_emit<GT, R>(a, tl, keys, state, scratch, a.scratch_bytes);
 }
 
