@@ -67,6 +67,16 @@ def measured_traffic():
     return d["dram_read_bytes_per_launch"] + d["dram_write_bytes_per_launch"]
 
 
+def ascending_order(order):
+    """The same visited block sets in ascending block order (the -1 padding
+    stays last): the visit order of the ablation without the HRM-first order."""
+    import torch
+    big = torch.iinfo(torch.int32).max
+    o = torch.where(order < 0, torch.full_like(order, big), order)
+    o = torch.sort(o, dim=-1).values
+    return torch.where(o == big, torch.full_like(o, -1), o)
+
+
 def rank_seed(cfg, rank, world):
     """Each rank prefills its own independent layer: distinct seeds for N > 1,
     the workload's own seed at N = 1."""
@@ -332,6 +342,27 @@ def run_cosa(args, rank, world, local_rank):
                                "stage2_budget": (vis - sk) / nqb_rows}
         extra["tau_sweep"] = sweep
         cosa.check(ws)
+        # visit-order ablation: the proxy's lists (HRM first, then by score) against the
+        # same block sets in ascending block order, at fixed tau
+        step(TAU)
+        torch.cuda.synchronize()
+        orders = {"hrm_first": sel["order"].clone(), "ascending": ascending_order(sel["order"])}
+        abl = {}
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for tau in (1e-4, 1e-3):
+            for name, ordr in orders.items():
+                cosa.attn(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], ordr, sel["count"], kmax,
+                          tau, ws, out=res)
+                e0.record(stream)
+                cosa.attn(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], ordr, sel["count"], kmax,
+                          tau, ws, out=res)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                vis = int(res["visited"].sum().item())
+                sk = int(res["skipped"].sum().item())
+                abl[f"{name}@{tau}"] = {"attn_ms": e0.elapsed_time(e1), "skip_ratio": sk / vis}
+        cosa.check(ws)
+        extra["order_ablation"] = abl
         # dense reference on the same B200: our OSK at budget 100% / tau 0, and torch SDPA (flash)
         ws_d, kmax_d = cosa.alloc_workspace(batch, 1.0)
         sel_d = cosa.proxy(batch, d["q"], d["k_pages"], d["page_table"], 1.0, kmax_d, ws_d)

@@ -120,6 +120,33 @@ def test_order_invariance_on_gpu():
     assert (a - b).abs().mean().item() <= gu.MEAN_ABS
 
 
+def ascending_rows(order, count):
+    """Each row's visited blocks in ascending block order (the -1 padding stays last)."""
+    o = order.copy()
+    for h in range(o.shape[0]):
+        for I in range(o.shape[1]):
+            o[h, I, :count[h, I]] = np.sort(o[h, I, :count[h, I]])
+    return o
+
+
+@pytest.mark.parametrize("name,tau", [("ragged_b128_p64", 1e-3), ("qwen_mix", 1e-2)])
+def test_attn_ascending_order_matches_oracle(name, tau):
+    """Visit-order ablation: the same block sets visited in ascending block order
+    (no HRM-first order) match the oracle run on that order, skip sets included."""
+    budget = 0.25
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], budget)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], budget, kmax, ws)
+    cnt = sel["count"].cpu().numpy()
+    asc = torch.from_numpy(ascending_rows(sel["order"].cpu().numpy(), cnt)).cuda()
+    res = gu.run_attn(d, dict(order=asc, count=sel["count"]), kmax, tau, ws)
+    r = oracle_proxy(name, budget)
+    ref = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size,
+                  ascending_rows(r["order"], r["count"]), r["count"], tau)
+    stats = gu.compare_attn(res, ref, w, tau, gu.all_units(w))
+    print(name, tau, stats)
+
+
 def test_repeated_calls_are_deterministic():
     d = device("qwen_mix")
     ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
