@@ -16,29 +16,32 @@
 //   Appendix C.2 (Algorithm A) and D.1 (b = 128 logical blocks, pages of any
 //        size b_p resolving a block; the vote reuses the on-chip row maxima).
 //
-// One CTA per (query head, q-block) tile, 320 threads, warp-specialised:
+// One CTA per (query head, q-block) tile, 320 threads, two CTAs per SM,
+// warp-specialised:
 //   warps 0-7  softmax: two threads per query row (TMEM lane), each owning
-//              half of the block's key columns.  tcgen05.ld of its half row,
-//              causal mask on the diagonal block, half-row max, the skip vote
-//              (a row votes to skip iff both of its halves lie below the
-//              threshold, so no exchange is needed: warp __all_sync + one
-//              256-thread named barrier), exp2 -> bf16 P written back into
-//              its own half of the S columns in TMEM, partial row sums, lazy
-//              rescaling of its half of O in TMEM, the epilogue O / l.
+//              half of the block's key columns, read 32 columns at a time.
+//              First pass: causal mask on the diagonal block, half-row max,
+//              the skip vote (a row votes to skip iff both of its halves lie
+//              below the threshold, so no exchange is needed: warp
+//              __all_sync + one 256-thread named barrier).  Second pass, if
+//              kept: exp2 -> bf16 P written back over the already-read S
+//              columns in TMEM, partial row sums; lazy rescaling of its half
+//              of O in TMEM; the epilogue O / l.
 //   warp 8     producer: page remap (order -> page_table) and TMA loads of the
-//              Q tile and of each block's K and V pages into 3-stage rings.
-//              Block and page ids are loaded two blocks ahead of the copies and
-//              lane u issues the boxes of page u; a block ending past the
-//              sequence is copied by hand with zero fill so no stray page slot
-//              reaches an MMA.
+//              Q tile and of each block's K and V pages into one K and one V
+//              slot.  Block and page ids are loaded two blocks ahead of the
+//              copies and lane u issues the boxes of page u; a block ending
+//              past the sequence is copied by hand with zero fill so no stray
+//              page slot reaches an MMA.
 //   warp 9     MMA issuer: S = Q K^T (M=128, N=b, K=d; both operands in shared
-//              memory) into one of three TMEM S buffers (block t uses t % 3),
-//              then O += P V (M=128, N=d, K=b) with P read from TMEM, unless
-//              the tile voted to skip; completion is signalled with
-//              tcgen05.commit.  S of block t+2 is issued right after P V of
-//              block t, a whole block ahead of the softmax warps.
+//              memory) into the TMEM S buffer, then O += P V (M=128, N=d,
+//              K=b) with P read from TMEM, unless the tile voted to skip;
+//              completion is signalled with tcgen05.commit.
+// Inside a CTA the chain is sequential (S, softmax, P V, next S); the second
+// CTA on the SM (98 KiB of shared memory, 256 TMEM columns and at most 96
+// registers per thread each) fills its gaps, prologue and epilogue included.
 // The tensor pipe executes one thread's MMAs in issue order, so P V of block
-// t-1 has read its P before S of block t+2 overwrites the same columns.
+// t has read its P before S of block t+1 overwrites the same columns.
 // Every wait is bounded; on expiry the CTA records COSA_ERR_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
 #include <cstdint>
@@ -57,7 +60,7 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr int kBQ = 128;          // query rows per tile (TMEM lanes)
-constexpr int kStages = 3;        // K and V ring depth
+constexpr int kStages = 1;        // K and V slots per CTA (two CTAs share an SM)
 constexpr uint32_t kDrainLimit = 1u << 22;
 constexpr float kRescaleLog2 = 8.0f;  // re-base O when the row max grows by > 2^8
 
@@ -65,7 +68,7 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[3];
+  uint64_t s_full[1];
   uint64_t p_full[2];   // softmax verdict (and P, if kept) for block t, by t & 1
   uint64_t o_done[2];   // P V of kept block c has completed, by c & 1
   uint64_t mma_drain;
@@ -88,10 +91,10 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_V + kStages * KV_BYTES;
   static constexpr int HALF = BK / 2;   // key columns per softmax thread
   static constexpr int KPH = HALF / 16; // K=16 MMA steps per half
-  // three S buffers (block t uses t % 3), so S of block t+2 can be issued
-  // right after P V of block t, while P of block t+1 still occupies its own
-  static constexpr int TMEM_O = 3 * BK;
-  static constexpr int TMEM_NEED = 3 * BK + D;
+  // one S buffer (P of block t overwrites it) and O: 256 columns for b = d = 128,
+  // so two CTAs share an SM's TMEM
+  static constexpr int TMEM_O = BK;
+  static constexpr int TMEM_NEED = BK + D;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                    : TMEM_NEED <= 256 ? 256 : 512;
   // Shared memory is padded so that the CTAs resident on one SM never ask
@@ -136,10 +139,10 @@ __device__ void manual_block_copy(unsigned char* stage, const __nv_bfloat16* poo
 
 }  // namespace
 
-// 10 warps put 3 warps on some SM sub-partitions, each with 16K registers,
-// which caps a thread at 168 registers.
+// Two CTAs of 10 warps put 5 warps on some SM sub-partitions, each with 16K
+// registers, which caps a thread at 96 registers.
 template <int D, int BK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     osk_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const OskArgs a) {
   using C = Cfg<D, BK>;
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_full[x], 1);
       mbar_init(&bars->v_empty[x], 1);
     }
-    for (int x = 0; x < 3; ++x) mbar_init(&bars->s_full[x], 1);
+    mbar_init(&bars->s_full[0], 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->p_full[x], kSoftmaxThreads);
       mbar_init(&bars->o_done[x], 1);
@@ -304,25 +307,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
       bool ok = mbar_wait(&bars->q_full, 0, a.wait_limit, abort, a.status, 0x20);
       int kept = 0;
-      // S = Q K^T of block t into S buffer t % 3
+      // S = Q K^T of block t into the S buffer
       auto issue_s = [&](int t) -> bool {
         const int slot = t % kStages, use = t / kStages;
         if (!mbar_wait(&bars->k_full[slot], use & 1, a.wait_limit, abort, a.status, 0x21)) return false;
         tc_fence_after();
-        const uint32_t d_s = tmem + (t % 3) * BK;
+        const uint32_t d_s = tmem;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t ad = sw128_desc(q_base + (ks >> 2) * (kBQ * 128) + (ks & 3) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(k_base + slot * C::KV_BYTES + (ks >> 2) * (BK * 128) + (ks & 3) * 32, 16, 1024);
           tc_mma_ss(d_s, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&bars->s_full[t % 3]);
+        tc_commit(&bars->s_full[0]);
         tc_commit(&bars->k_empty[slot]);
         return true;
       };
-      if (ok && n > 0) ok = issue_s(0);
-      if (ok && n > 1) ok = issue_s(1);
       for (int u = 0; u < n && ok; ++u) {
+        // S of block u takes the buffer whose P V (block u-1) was issued just before
+        ok = issue_s(u);
+        if (!ok) break;
         const int vslot = u % kStages, vuse = u / kStages;
         ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, a.wait_limit, abort, a.status, 0x23);
         if (ok) ok = mbar_wait(&bars->v_full[vslot], vuse & 1, a.wait_limit, abort, a.status, 0x24);
@@ -330,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[u & 1]);
         if (!skip) {
-          const uint32_t p_tmem = tmem + (u % 3) * BK;
+          const uint32_t p_tmem = tmem;
           const uint32_t d_o = tmem + C::TMEM_O;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
@@ -346,8 +350,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           mbar_arrive(&bars->v_empty[vslot]);
         }
-        // S of block u+2 reuses the buffer of block u-1, whose P V was issued above
-        if (u + 2 < n) ok = issue_s(u + 2);
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
       tc_commit(&bars->mma_drain);
@@ -368,36 +370,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     int j_next = __ldg(ord);
     for (int t = 0; t < n; ++t) {
       const int sb = t & 1;
-      const int sbuf = t % 3;
-      const uint32_t s_cols = lane_base + sbuf * BK + col0;
+      const uint32_t s_cols = lane_base + col0;
       const int j = j_next;
       if (t + 1 < n) j_next = __ldg(ord + t + 1);
-      bool ok = mbar_wait(&bars->s_full[sbuf], (t / 3) & 1, a.wait_limit, abort, a.status, 0x30);
+      bool ok = mbar_wait(&bars->s_full[0], t & 1, a.wait_limit, abort, a.status, 0x30);
       ok = __all_sync(0xffffffffu, ok) && !aborted;
-      float sv[C::HALF];
+      // first pass: the half-row max, 32 columns at a time
+      float mx = -INFINITY;
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < C::HALF / 32; ++c) tmem_ld32(s_cols + c * 32, sv + c * 32);
-        tc_wait_ld();
-      }
-      // causal mask (only the diagonal block, or a block past it, can hide keys):
-      // key k of block j is visible to row r iff j*b + k <= i*b + r
-      if (j >= i) {
-        const int lim = r - (j - i) * b - col0;
+        for (int c = 0; c < C::HALF / 32; ++c) {
+          float sc[32];
+          tmem_ld32(s_cols + c * 32, sc);
+          tc_wait_ld();
+          // causal mask (only the diagonal block, or a block past it, can hide keys):
+          // key k of block j is visible to row r iff j*b + k <= i*b + r
+          if (j >= i) {
+            const int lim = r - (j - i) * b - col0 - c * 32;
 #pragma unroll
-        for (int k = 0; k < C::HALF; ++k)
-          if (k > lim) sv[k] = -INFINITY;
-      }
-      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+            for (int k = 0; k < 32; ++k)
+              if (k > lim) sc[k] = -INFINITY;
+          }
+          float mx0 = sc[0], mx1 = sc[1], mx2 = sc[2], mx3 = sc[3];
 #pragma unroll
-      for (int k = 4; k < C::HALF; k += 4) {
-        mx0 = fmaxf(mx0, sv[k]);
-        mx1 = fmaxf(mx1, sv[k + 1]);
-        mx2 = fmaxf(mx2, sv[k + 2]);
-        mx3 = fmaxf(mx3, sv[k + 3]);
+          for (int k = 4; k < 32; k += 4) {
+            mx0 = fmaxf(mx0, sc[k]);
+            mx1 = fmaxf(mx1, sc[k + 1]);
+            mx2 = fmaxf(mx2, sc[k + 2]);
+            mx3 = fmaxf(mx3, sc[k + 3]);
+          }
+          mx = fmaxf(mx, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+        }
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
       const float m_half = (row_valid && mx != -INFINITY) ? mx * sl2 : -INFINITY;
       const float gap = (m_half == -INFINITY) ? -INFINITY : m_half - m;
       const bool votes_skip = !row_valid || gap < a.log2_tau;
@@ -438,17 +443,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = exp2(s * log2e/sqrt(d) - ref) in bf16; partial row sum of the fp32 values.
       // Rows past the sequence end need no masking here: a row of P only feeds the
       // same row of O, and those rows of O are never written out.
-      uint32_t pk[C::HALF / 2];
       float2 ls = make_float2(0.0f, 0.0f);
       const float nb = (new_ref == -INFINITY) ? 0.0f : -new_ref;
       const float2 sl2x2 = make_float2(sl2, sl2), nbx2 = make_float2(nb, nb);
+      // second pass over the S columns, 32 at a time (registers are capped at 96 with two
+      // CTAs per SM): P of chunk c goes to columns [16c, 16c + 16) of this thread's
+      // half, all already read
 #pragma unroll
-      for (int e = 0; e < C::HALF / 2; ++e) {
-        // two logits per packed fp32 FMA, two sums per packed add
-        const float2 x = fma_f32x2(make_float2(sv[2 * e], sv[2 * e + 1]), sl2x2, nbx2);
-        const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        pk[e] = pack_bf16x2(pv.x, pv.y);
-        ls = add_f32x2(ls, pv);
+      for (int c = 0; c < C::HALF / 32; ++c) {
+        float sc[32];
+        tmem_ld32(s_cols + c * 32, sc);
+        tc_wait_ld();
+        if (j >= i) {
+          const int lim = r - (j - i) * b - col0 - c * 32;
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (k > lim) sc[k] = -INFINITY;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          // two logits per packed fp32 FMA, two sums per packed add
+          const float2 x = fma_f32x2(make_float2(sc[2 * e], sc[2 * e + 1]), sl2x2, nbx2);
+          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          pk[e] = pack_bf16x2(pv.x, pv.y);
+          ls = add_f32x2(ls, pv);
+        }
+        tmem_st16(s_cols + c * 16, pk);
       }
       const float ls0 = ls.x, ls1 = ls.y;
       if (rescale) {
@@ -473,12 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mref = new_ref;
       m = m_new;
       l += ls0 + ls1;
-      // P over this thread's own (already read) S columns, packed bf16 pairs
-      if constexpr (C::HALF == 64) {
-        tmem_st32(s_cols, reinterpret_cast<const float*>(pk));
-      } else {
-        tmem_st16(s_cols, pk);
-      }
       tc_wait_st();
       tc_fence_before();
       if (tid == 0) {
