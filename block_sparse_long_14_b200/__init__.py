@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "Batch", "CosaError", "alloc_workspace", "attn", "check", "lib", "proxy", "remap",
-    "set_wait_limit", "workspace_size", "LIB_PATH",
+    "set_wait_limit", "tau_from_delta", "workspace_size", "LIB_PATH",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -223,6 +223,24 @@ def attn(batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int,
                           workspace.numel(), _stream())
     _check(rc, "cosa_attn")
     return res
+
+
+def tau_from_delta(delta: float, seq_len: int) -> float:
+    """The length-adaptive skip threshold of the paper (§5.1 "Hyperparameters",
+    Appendix D.1 "CoSA settings"; the operating points there are delta = 2000
+    for Qwen3-8B and 200 for Llama-3.1-8B): tau = delta / N with N the
+    sequence length in tokens; delta = -1 turns the in-kernel skip off
+    (tau = 0).  A ragged batch
+    with one delta has one tau per sequence; `attn` takes one tau per call, so
+    such a batch is attended per sequence, or with the tau of a chosen N."""
+    if delta == -1:
+        return 0.0
+    if not (delta >= 0 and seq_len > 0):
+        raise ValueError(f"delta must be -1 or >= 0 and seq_len > 0 (got {delta}, {seq_len})")
+    tau = float(delta) / float(seq_len)
+    if not tau < 1.0:
+        raise ValueError(f"delta / seq_len = {tau} is not a threshold in [0, 1)")
+    return tau
 
 
 def check(workspace):
