@@ -20,7 +20,7 @@ import os
 import torch
 
 __all__ = [
-    "Batch", "CosaError", "alloc_workspace", "attn", "check", "lib", "proxy", "remap",
+    "Batch", "CosaError", "alloc_workspace", "attn", "attn_delta", "check", "lib", "proxy", "remap",
     "set_wait_limit", "tau_from_delta", "workspace_size", "LIB_PATH",
 ]
 
@@ -59,6 +59,8 @@ _SIGS = {
     "cosa_remap": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, ctypes.c_int32, _P, _P]),
     "cosa_attn": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_float,
                                  _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "cosa_attn_delta": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, _P, _P, _P, ctypes.c_int32,
+                                       ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "cosa_sync_status": (ctypes.c_int, [_P, _P]),
     "cosa_debug_set_wait_limit": (None, [ctypes.c_uint32]),
     "cosa_error_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -202,9 +204,8 @@ def remap(batch: Batch, page_table, order, count, kmax: int, pages=None):
     return pages
 
 
-def attn(batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int, tau: float, workspace,
-         out=None, skipbits: bool = False):
-    """OSK attention.  Returns dict(out, visited, skipped[, skipbits])."""
+def _attn(entry, batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int, thr: float, workspace,
+          out, skipbits: bool):
     H, N = batch.num_q_heads, batch.total_qblocks
     dev = q.device
     res = out if out is not None else dict(
@@ -214,15 +215,29 @@ def attn(batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int,
     if skipbits and "skipbits" not in res:
         res["skipbits"] = torch.empty((H, N, kmax), dtype=torch.uint8, device=dev)
     sb = res.get("skipbits") if skipbits else None
-    rc = _lib().cosa_attn(ctypes.byref(batch.c), _ptr(q, torch.bfloat16, "q"), _ptr(k_pages, torch.bfloat16, "k_pages"),
-                          _ptr(v_pages, torch.bfloat16, "v_pages"), _ptr(page_table, torch.int32, "page_table"),
-                          _ptr(order, torch.int32, "order"), _ptr(count, torch.int32, "count"), int(kmax),
-                          ctypes.c_float(tau), _ptr(res["out"], torch.bfloat16, "out"),
-                          _ptr(res["visited"], torch.int32, "visited"), _ptr(res["skipped"], torch.int32, "skipped"),
-                          _ptr(sb, torch.uint8, "skipbits"), _ptr(workspace, torch.uint8, "workspace"),
-                          workspace.numel(), _stream())
-    _check(rc, "cosa_attn")
+    rc = getattr(_lib(), entry)(
+        ctypes.byref(batch.c), _ptr(q, torch.bfloat16, "q"), _ptr(k_pages, torch.bfloat16, "k_pages"),
+        _ptr(v_pages, torch.bfloat16, "v_pages"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(order, torch.int32, "order"), _ptr(count, torch.int32, "count"), int(kmax), ctypes.c_float(thr),
+        _ptr(res["out"], torch.bfloat16, "out"), _ptr(res["visited"], torch.int32, "visited"),
+        _ptr(res["skipped"], torch.int32, "skipped"), _ptr(sb, torch.uint8, "skipbits"),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream())
+    _check(rc, entry)
     return res
+
+
+def attn(batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int, tau: float, workspace,
+         out=None, skipbits: bool = False):
+    """OSK attention with one skip threshold tau.  Returns dict(out, visited, skipped[, skipbits])."""
+    return _attn("cosa_attn", batch, q, k_pages, v_pages, page_table, order, count, kmax, tau, workspace, out,
+                 skipbits)
+
+
+def attn_delta(batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int, delta: float, workspace,
+               out=None, skipbits: bool = False):
+    """OSK attention with tau_s = delta / L_s per sequence (delta = -1: no skip)."""
+    return _attn("cosa_attn_delta", batch, q, k_pages, v_pages, page_table, order, count, kmax, delta, workspace,
+                 out, skipbits)
 
 
 def tau_from_delta(delta: float, seq_len: int) -> float:
@@ -230,9 +245,8 @@ def tau_from_delta(delta: float, seq_len: int) -> float:
     Appendix D.1 "CoSA settings"; the operating points there are delta = 2000
     for Qwen3-8B and 200 for Llama-3.1-8B): tau = delta / N with N the
     sequence length in tokens; delta = -1 turns the in-kernel skip off
-    (tau = 0).  A ragged batch
-    with one delta has one tau per sequence; `attn` takes one tau per call, so
-    such a batch is attended per sequence, or with the tau of a chosen N."""
+    (tau = 0).  `attn_delta` applies the same mapping on the device, one
+    tau per sequence of a ragged batch."""
     if delta == -1:
         return 0.0
     if not (delta >= 0 and seq_len > 0):

@@ -264,17 +264,20 @@ int cosa_remap(const cosa_shape_t* shape, const int32_t* page_table, const int32
   return launch_remap(ra, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COSA_OK : COSA_ERR_CUDA;
 }
 
-int cosa_attn(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
-              const int32_t* page_table, const int32_t* order, const int32_t* count, int32_t kmax, float tau,
-              void* out, int32_t* visited, int32_t* skipped, uint8_t* skipbits, void* workspace, size_t ws_bytes,
-              cosa_stream_t stream) {
+namespace {
+
+// The shared body of cosa_attn and cosa_attn_delta: tau_per_seq selects
+// between one threshold (log2_tau) and tau_s = delta / L_s (log2_delta).
+int attn_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
+              const int32_t* page_table, const int32_t* order, const int32_t* count, int32_t kmax, float log2_tau,
+              int tau_per_seq, float log2_delta, void* out, int32_t* visited, int32_t* skipped, uint8_t* skipbits,
+              void* workspace, size_t ws_bytes, cosa_stream_t stream) {
   int rc = check_shape(shape);
   if (rc != COSA_OK) return rc;
   if (q == nullptr || k_pages == nullptr || v_pages == nullptr || page_table == nullptr || order == nullptr ||
       count == nullptr || out == nullptr || visited == nullptr || skipped == nullptr || workspace == nullptr ||
       kmax < 1)
     return COSA_ERR_INVALID_ARG;
-  if (!(tau >= 0.0f && tau < 1.0f)) return COSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return COSA_ERR_INVALID_ARG;
@@ -321,10 +324,34 @@ int cosa_attn(const cosa_shape_t* shape, const void* q, const void* k_pages, con
   oa.nqb_total = shape->total_qblocks;
   oa.kmax = kmax;
   oa.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  oa.log2_tau = tau > 0.0f ? static_cast<float>(std::log2(static_cast<double>(tau))) : -INFINITY;
+  oa.log2_tau = log2_tau;
+  oa.tau_per_seq = tau_per_seq;
+  oa.log2_delta = log2_delta;
   oa.wait_limit = g_wait_limit.load();
   return launch_osk(oa, qmap, kmap, vmap, D, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COSA_OK
                                                                                                       : COSA_ERR_CUDA;
+}
+
+}  // namespace
+
+int cosa_attn(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
+              const int32_t* page_table, const int32_t* order, const int32_t* count, int32_t kmax, float tau,
+              void* out, int32_t* visited, int32_t* skipped, uint8_t* skipbits, void* workspace, size_t ws_bytes,
+              cosa_stream_t stream) {
+  if (!(tau >= 0.0f && tau < 1.0f)) return COSA_ERR_INVALID_ARG;
+  const float log2_tau = tau > 0.0f ? static_cast<float>(std::log2(static_cast<double>(tau))) : -INFINITY;
+  return attn_impl(shape, q, k_pages, v_pages, page_table, order, count, kmax, log2_tau, 0, -INFINITY, out, visited,
+                   skipped, skipbits, workspace, ws_bytes, stream);
+}
+
+int cosa_attn_delta(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* order, const int32_t* count, int32_t kmax, float delta,
+                    void* out, int32_t* visited, int32_t* skipped, uint8_t* skipbits, void* workspace,
+                    size_t ws_bytes, cosa_stream_t stream) {
+  if (!(delta == -1.0f || (delta > 0.0f && std::isfinite(delta)))) return COSA_ERR_INVALID_ARG;
+  const float log2_delta = delta > 0.0f ? static_cast<float>(std::log2(static_cast<double>(delta))) : -INFINITY;
+  return attn_impl(shape, q, k_pages, v_pages, page_table, order, count, kmax, -INFINITY, 1, log2_delta, out, visited,
+                   skipped, skipbits, workspace, ws_bytes, stream);
 }
 
 int cosa_sync_status(void* workspace, cosa_stream_t stream) {

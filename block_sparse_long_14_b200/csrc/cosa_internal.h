@@ -68,6 +68,8 @@ struct OskArgs {
   int nqb_total, kmax;
   float scale_log2;  // log2(e) / sqrt(d)
   float log2_tau;    // log2(tau), -inf for tau = 0
+  int tau_per_seq;   // 1: tau_s = delta / L_s per sequence, log2(tau_s) = log2_delta - log2(L_s)
+  float log2_delta;  // log2(delta), -inf when the skip is off
   uint32_t wait_limit;
 };
 

@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int b = a.block_size;
   const int nrows = min(b, L - i * b);
   const int nkb = (L + b - 1) / b;
+  // skip threshold of this sequence: one tau, or tau_s = delta / L_s
+  const float log2_tau = a.tau_per_seq ? a.log2_delta - log2f(static_cast<float>(L)) : a.log2_tau;
   const long row_id = static_cast<long>(h) * a.nqb_total + I;
   int n = __ldg(a.count + row_id);
   if (n < 0 || n > a.kmax) {
@@ -405,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       const float m_half = (row_valid && mx != -INFINITY) ? mx * sl2 : -INFINITY;
       const float gap = (m_half == -INFINITY) ? -INFINITY : m_half - m;
-      const bool votes_skip = !row_valid || gap < a.log2_tau;
+      const bool votes_skip = !row_valid || gap < log2_tau;
       const bool wskip = __all_sync(0xffffffffu, votes_skip);
       if (lane == 0) bars->vote[sb][warp] = (ok ? 0 : 2) | (wskip ? 1 : 0);
       bars->half_max[sb][half][r] = m_half;

@@ -212,6 +212,20 @@ COSA_API int cosa_attn(const cosa_shape_t* shape, const void* q, const void* k_p
               uint8_t* skipbits, void* workspace, size_t ws_bytes, cosa_stream_t stream);
 
 /*
+ * OSK attention with the pages' length-adaptive threshold (§5.1
+ * "Hyperparameters", Appendix D.1 "CoSA settings"): each sequence s of the
+ * batch uses tau_s = delta / L_s, L_s its length in tokens, computed on the
+ * device from cu_seqlens.  delta = -1 turns the skip off (tau = 0 for every
+ * sequence); otherwise delta must be > 0.  tau_s >= 1 (a sequence shorter
+ * than delta) is applied as written: the skip test compares against
+ * ln(tau_s) >= 0.  All other arguments, outputs and errors as cosa_attn.
+ */
+COSA_API int cosa_attn_delta(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
+                    const int32_t* page_table, const int32_t* order, const int32_t* count,
+                    int32_t kmax, float delta, void* out, int32_t* visited, int32_t* skipped,
+                    uint8_t* skipbits, void* workspace, size_t ws_bytes, cosa_stream_t stream);
+
+/*
  * Synchronise `stream`, read and clear the workspace's status word.
  * Returns COSA_OK, COSA_ERR_TIMEOUT, COSA_ERR_DEVICE or COSA_ERR_CUDA.
  */

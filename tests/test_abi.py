@@ -106,3 +106,19 @@ def test_null_pointers_rejected_before_launch(lib):
     assert rc == 1
     rc = lib.cosa_remap(ctypes.byref(sh), None, None, None, 52, None, None)
     assert rc == 1
+
+
+@pytest.mark.parametrize("delta", [0.0, -0.5, -2.0, float("nan"), float("inf")])
+def test_attn_delta_rejects_bad_delta(lib, delta):
+    sh = _shape()
+    rc = lib.cosa_attn_delta(ctypes.byref(sh), None, None, None, None, None, None, 52, ctypes.c_float(delta), None,
+                             None, None, None, None, 0, None)
+    assert rc == 1
+
+
+def test_attn_rejects_tau_outside_unit_interval(lib):
+    sh = _shape()
+    for tau in (-1e-3, 1.0, 2.0, float("nan")):
+        rc = lib.cosa_attn(ctypes.byref(sh), None, None, None, None, None, None, 52, ctypes.c_float(tau), None,
+                           None, None, None, None, 0, None)
+        assert rc == 1

@@ -147,6 +147,32 @@ def test_attn_ascending_order_matches_oracle(name, tau):
     print(name, tau, stats)
 
 
+@pytest.mark.parametrize("name,delta", [("ragged_b128_p64", 20.0), ("short_seqs", 2.0), ("ragged_b128_p64", -1.0)])
+def test_attn_delta_matches_oracle_per_sequence(name, delta):
+    """tau_s = delta / L_s per sequence (the pages' length-adaptive threshold),
+    against the oracle run sequence by sequence with that sequence's tau."""
+    budget = 0.25
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], budget)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], budget, kmax, ws)
+    res = cosa.attn_delta(d["batch"], d["q"], d["k_pages"], d["v_pages"], d["page_table"], sel["order"],
+                          sel["count"], kmax, delta, ws, skipbits=True)
+    cosa.check(ws)
+    r = oracle_proxy(name, budget)
+    b = w.block_size
+    nqb = [(L + b - 1) // b for L in w.seqlens]
+    qb0 = np.concatenate([[0], np.cumsum(nqb)])
+    for s_i, L in enumerate(w.seqlens):
+        tau = 0.0 if delta == -1.0 else delta / L
+        units = [(h, I) for h in range(w.num_q_heads) for I in range(qb0[s_i], qb0[s_i + 1])]
+        ref = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size,
+                      r["order"], r["count"], tau, units=units)
+        stats = gu.compare_attn(res, ref, w, tau, units)
+        print(name, delta, s_i, L, tau, stats)
+    if delta == -1.0:
+        assert int(res["skipped"].sum()) == 0
+
+
 def test_repeated_calls_are_deterministic():
     d = device("qwen_mix")
     ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
