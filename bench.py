@@ -77,6 +77,27 @@ def ascending_order(order):
     return torch.where(o == big, torch.full_like(o, -1), o)
 
 
+def masked_full_lists(order, count, seqlens, block_size):
+    """For the logical-mask ablation: every row's list becomes all its causal
+    blocks 0..i in ascending order, with keep = 1 on the blocks the proxy
+    selected.  Returns (order_full, count_full, keep, kmax_full)."""
+    import torch
+    H, N, kmax = order.shape
+    dev = order.device
+    nqb = [(L + block_size - 1) // block_size for L in seqlens]
+    qb_local = torch.cat([torch.arange(n, dtype=torch.int32) for n in nqb]).to(dev)   # [N]
+    kmax_full = max(nqb)
+    ar = torch.arange(kmax_full, dtype=torch.int32, device=dev)
+    full = ar.expand(H, N, kmax_full).clone()
+    full[ar.view(1, 1, -1).expand(H, N, -1) > qb_local.view(1, -1, 1).expand(H, -1, kmax_full)] = -1
+    count_full = (qb_local + 1).view(1, -1).expand(H, N).contiguous()
+    valid = torch.arange(kmax, device=dev).view(1, 1, -1) < count.view(H, N, 1)
+    idx = torch.where(valid, order.long(), torch.full_like(order, kmax_full).long())
+    keep = torch.zeros((H, N, kmax_full + 1), dtype=torch.uint8, device=dev)
+    keep.scatter_(2, idx, valid.to(torch.uint8))
+    return full.contiguous(), count_full, keep[:, :, :kmax_full].contiguous(), kmax_full
+
+
 def rank_seed(cfg, rank, world):
     """Each rank prefills its own independent layer: distinct seeds for N > 1,
     the workload's own seed at N = 1."""
@@ -362,6 +383,24 @@ def run_cosa(args, rank, world, local_rank):
                 sk = int(res["skipped"].sum().item())
                 abl[f"{name}@{tau}"] = {"attn_ms": e0.elapsed_time(e1), "skip_ratio": sk / vis}
         cosa.check(ws)
+        # logical-mask execution of the ascending run: every causal block is walked, the
+        # unselected ones passed over with a mask check (physical jumping vs a mask loop)
+        o_full, c_full, keep, kmax_full = masked_full_lists(sel["order"], sel["count"], w.seqlens, w.block_size)
+        ws_m, _ = cosa.alloc_workspace(batch, 1.0)
+        for tau in (1e-4, 1e-3):
+            cosa.attn_masked(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], o_full, c_full, kmax_full,
+                             keep, tau, ws_m, out=res)
+            e0.record(stream)
+            cosa.attn_masked(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], o_full, c_full, kmax_full,
+                             keep, tau, ws_m, out=res)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            vis = int(res["visited"].sum().item())
+            sk = int(res["skipped"].sum().item())
+            abl[f"mask_loop@{tau}"] = {"attn_ms": e0.elapsed_time(e1), "skip_ratio": sk / vis,
+                                       "entries_walked": int(c_full.sum().item())}
+        cosa.check(ws_m)
+        del o_full, c_full, keep, ws_m
         extra["order_ablation"] = abl
         # dense reference on the same B200: our OSK at budget 100% / tau 0, and torch SDPA (flash)
         ws_d, kmax_d = cosa.alloc_workspace(batch, 1.0)

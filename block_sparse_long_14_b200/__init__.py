@@ -20,7 +20,7 @@ import os
 import torch
 
 __all__ = [
-    "Batch", "CosaError", "alloc_workspace", "attn", "attn_delta", "check", "lib", "proxy", "remap",
+    "Batch", "CosaError", "alloc_workspace", "attn", "attn_delta", "attn_masked", "check", "lib", "proxy", "remap",
     "set_wait_limit", "tau_from_delta", "workspace_size", "LIB_PATH",
 ]
 
@@ -61,6 +61,8 @@ _SIGS = {
                                  _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "cosa_attn_delta": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, _P, _P, _P, ctypes.c_int32,
                                        ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "cosa_attn_masked": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P,
+                                        ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "cosa_sync_status": (ctypes.c_int, [_P, _P]),
     "cosa_debug_set_wait_limit": (None, [ctypes.c_uint32]),
     "cosa_error_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -205,7 +207,7 @@ def remap(batch: Batch, page_table, order, count, kmax: int, pages=None):
 
 
 def _attn(entry, batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int, thr: float, workspace,
-          out, skipbits: bool):
+          out, skipbits: bool, keep=None):
     H, N = batch.num_q_heads, batch.total_qblocks
     dev = q.device
     res = out if out is not None else dict(
@@ -215,10 +217,13 @@ def _attn(entry, batch: Batch, q, k_pages, v_pages, page_table, order, count, km
     if skipbits and "skipbits" not in res:
         res["skipbits"] = torch.empty((H, N, kmax), dtype=torch.uint8, device=dev)
     sb = res.get("skipbits") if skipbits else None
+    head = [ctypes.byref(batch.c), _ptr(q, torch.bfloat16, "q"), _ptr(k_pages, torch.bfloat16, "k_pages"),
+            _ptr(v_pages, torch.bfloat16, "v_pages"), _ptr(page_table, torch.int32, "page_table"),
+            _ptr(order, torch.int32, "order"), _ptr(count, torch.int32, "count"), int(kmax)]
+    if keep is not None:
+        head.append(_ptr(keep, torch.uint8, "keep"))
     rc = getattr(_lib(), entry)(
-        ctypes.byref(batch.c), _ptr(q, torch.bfloat16, "q"), _ptr(k_pages, torch.bfloat16, "k_pages"),
-        _ptr(v_pages, torch.bfloat16, "v_pages"), _ptr(page_table, torch.int32, "page_table"),
-        _ptr(order, torch.int32, "order"), _ptr(count, torch.int32, "count"), int(kmax), ctypes.c_float(thr),
+        *head, ctypes.c_float(thr),
         _ptr(res["out"], torch.bfloat16, "out"), _ptr(res["visited"], torch.int32, "visited"),
         _ptr(res["skipped"], torch.int32, "skipped"), _ptr(sb, torch.uint8, "skipbits"),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream())
@@ -238,6 +243,15 @@ def attn_delta(batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax
     """OSK attention with tau_s = delta / L_s per sequence (delta = -1: no skip)."""
     return _attn("cosa_attn_delta", batch, q, k_pages, v_pages, page_table, order, count, kmax, delta, workspace,
                  out, skipbits)
+
+
+def attn_masked(batch: Batch, q, k_pages, v_pages, page_table, order, count, kmax: int, keep, tau: float,
+                workspace, out=None, skipbits: bool = False):
+    """OSK attention in logical-mask execution: every list entry is walked and
+    only those with keep[h, I, t] != 0 are computed (the ablation of physical
+    jumping over pages)."""
+    return _attn("cosa_attn_masked", batch, q, k_pages, v_pages, page_table, order, count, kmax, tau, workspace,
+                 out, skipbits, keep=keep)
 
 
 def tau_from_delta(delta: float, seq_len: int) -> float:

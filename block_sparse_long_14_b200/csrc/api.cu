@@ -270,8 +270,8 @@ namespace {
 // between one threshold (log2_tau) and tau_s = delta / L_s (log2_delta).
 int attn_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
               const int32_t* page_table, const int32_t* order, const int32_t* count, int32_t kmax, float log2_tau,
-              int tau_per_seq, float log2_delta, void* out, int32_t* visited, int32_t* skipped, uint8_t* skipbits,
-              void* workspace, size_t ws_bytes, cosa_stream_t stream) {
+              int tau_per_seq, float log2_delta, const uint8_t* keep, void* out, int32_t* visited, int32_t* skipped,
+              uint8_t* skipbits, void* workspace, size_t ws_bytes, cosa_stream_t stream) {
   int rc = check_shape(shape);
   if (rc != COSA_OK) return rc;
   if (q == nullptr || k_pages == nullptr || v_pages == nullptr || page_table == nullptr || order == nullptr ||
@@ -313,6 +313,7 @@ int attn_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, con
   oa.visited = visited;
   oa.skipped = skipped;
   oa.skipbits = skipbits;
+  oa.keep = keep;
   oa.status = reinterpret_cast<Status*>(workspace);
   oa.batch = shape->batch;
   oa.num_q_heads = Hq;
@@ -340,8 +341,19 @@ int cosa_attn(const cosa_shape_t* shape, const void* q, const void* k_pages, con
               cosa_stream_t stream) {
   if (!(tau >= 0.0f && tau < 1.0f)) return COSA_ERR_INVALID_ARG;
   const float log2_tau = tau > 0.0f ? static_cast<float>(std::log2(static_cast<double>(tau))) : -INFINITY;
-  return attn_impl(shape, q, k_pages, v_pages, page_table, order, count, kmax, log2_tau, 0, -INFINITY, out, visited,
-                   skipped, skipbits, workspace, ws_bytes, stream);
+  return attn_impl(shape, q, k_pages, v_pages, page_table, order, count, kmax, log2_tau, 0, -INFINITY, nullptr, out,
+                   visited, skipped, skipbits, workspace, ws_bytes, stream);
+}
+
+int cosa_attn_masked(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
+                     const int32_t* page_table, const int32_t* order, const int32_t* count, int32_t kmax,
+                     const uint8_t* keep, float tau, void* out, int32_t* visited, int32_t* skipped,
+                     uint8_t* skipbits, void* workspace, size_t ws_bytes, cosa_stream_t stream) {
+  if (keep == nullptr) return COSA_ERR_INVALID_ARG;
+  if (!(tau >= 0.0f && tau < 1.0f)) return COSA_ERR_INVALID_ARG;
+  const float log2_tau = tau > 0.0f ? static_cast<float>(std::log2(static_cast<double>(tau))) : -INFINITY;
+  return attn_impl(shape, q, k_pages, v_pages, page_table, order, count, kmax, log2_tau, 0, -INFINITY, keep, out,
+                   visited, skipped, skipbits, workspace, ws_bytes, stream);
 }
 
 int cosa_attn_delta(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
@@ -350,8 +362,8 @@ int cosa_attn_delta(const cosa_shape_t* shape, const void* q, const void* k_page
                     size_t ws_bytes, cosa_stream_t stream) {
   if (!(delta == -1.0f || (delta > 0.0f && std::isfinite(delta)))) return COSA_ERR_INVALID_ARG;
   const float log2_delta = delta > 0.0f ? static_cast<float>(std::log2(static_cast<double>(delta))) : -INFINITY;
-  return attn_impl(shape, q, k_pages, v_pages, page_table, order, count, kmax, -INFINITY, 1, log2_delta, out, visited,
-                   skipped, skipbits, workspace, ws_bytes, stream);
+  return attn_impl(shape, q, k_pages, v_pages, page_table, order, count, kmax, -INFINITY, 1, log2_delta, nullptr, out,
+                   visited, skipped, skipbits, workspace, ws_bytes, stream);
 }
 
 int cosa_sync_status(void* workspace, cosa_stream_t stream) {

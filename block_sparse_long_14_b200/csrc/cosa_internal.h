@@ -63,6 +63,7 @@ struct OskArgs {
   int32_t* visited;
   int32_t* skipped;
   uint8_t* skipbits;
+  const uint8_t* keep;  // nullable: list entry t is computed only where keep[row, t] != 0
   Status* status;
   int batch, num_q_heads, num_kv_heads, block_size, page_size, max_pages_per_seq, num_pages;
   int nqb_total, kmax;

@@ -185,6 +185,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     n = n < 0 ? 0 : a.kmax;
   }
   const int32_t* ord = a.order + row_id * a.kmax;
+  // logical-mask execution: entry t of the list is computed only where keep != 0
+  const uint8_t* keep_row = a.keep != nullptr ? a.keep + row_id * a.kmax : nullptr;
   const int32_t* pt_row = a.page_table + static_cast<long>(s) * a.max_pages_per_seq;
 
   if (tid == kProducerWarp * 32) {
@@ -249,8 +251,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     int j_n = block_id(1);
     int pg_n = page_of(j_n);
     int j_nn = block_id(2);
+    int ncopy = 0;   // entries copied so far (all of them, unless a keep mask passes some over)
     for (int t = 0; t < n && ok; ++t) {
-      const int slot = t % kStages, use = t / kStages;
+      if (keep_row != nullptr && __ldg(keep_row + t) == 0) {
+        j_c = j_n;
+        pg_c = pg_n;
+        j_n = j_nn;
+        pg_n = page_of(j_nn);
+        j_nn = block_id(t + 3);
+        continue;
+      }
+      const int slot = ncopy % kStages, use = ncopy / kStages;
       int j = j_c;
       const int page = pg_c;
       bool jvalid = (j >= 0 && j < nkb);
@@ -289,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (kvsel == 0) k_armed[slot] = use; else v_armed[slot] = use;
       }
+      ++ncopy;
       j_c = j_n;
       pg_c = pg_n;
       j_n = j_nn;
@@ -325,7 +337,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_commit(&bars->k_empty[slot]);
         return true;
       };
-      for (int u = 0; u < n && ok; ++u) {
+      for (int t = 0, u = 0; t < n && ok; ++t) {
+        if (keep_row != nullptr && __ldg(keep_row + t) == 0) continue;
         // S of block u takes the buffer whose P V (block u-1) was issued just before
         ok = issue_s(u);
         if (!ok) break;
@@ -352,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         } else {
           mbar_arrive(&bars->v_empty[vslot]);
         }
+        ++u;
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
       tc_commit(&bars->mma_drain);
@@ -370,12 +384,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     int n_pv = 0, nskip = 0;
     bool aborted = false;
     int j_next = __ldg(ord);
+    int ncomp = 0;   // entries computed so far
     for (int t = 0; t < n; ++t) {
-      const int sb = t & 1;
-      const uint32_t s_cols = lane_base + col0;
       const int j = j_next;
       if (t + 1 < n) j_next = __ldg(ord + t + 1);
-      bool ok = mbar_wait(&bars->s_full[0], t & 1, a.wait_limit, abort, a.status, 0x30);
+      if (keep_row != nullptr && __ldg(keep_row + t) == 0) {
+        if (tid == 0 && a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 0;
+        continue;
+      }
+      const int sb = ncomp & 1;
+      ++ncomp;
+      const uint32_t s_cols = lane_base + col0;
+      bool ok = mbar_wait(&bars->s_full[0], sb, a.wait_limit, abort, a.status, 0x30);
       ok = __all_sync(0xffffffffu, ok) && !aborted;
       // first pass: the half-row max, 32 columns at a time
       float mx = -INFINITY;
@@ -509,14 +529,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = !aborted && n_pv >= 1;
     if (ok) ok = mbar_wait(&bars->o_done[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status, 0x32);
     ok = __all_sync(0xffffffffu, ok);
-    float (*half_l)[kBQ] = bars->half_max[n & 1];   // idle since the barrier of block n-1
+    float (*half_l)[kBQ] = bars->half_max[ncomp & 1];   // idle since the barrier of the last computed block
     half_l[half][r] = l;
     if (lane == 0) bars->vote_end[warp] = ok ? 1 : 0;
     named_bar_sync(1, kSoftmaxThreads);
     int all_ok = 1;
 #pragma unroll
     for (int w = 0; w < kSoftmaxWarps; ++w) all_ok &= bars->vote_end[w];
-    if (all_ok) {
+    if (ncomp == 0) {
+      // a keep mask that leaves nothing of the row: zero output, like an empty list
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(a.out + ((static_cast<long>(tok0) + i * b + r) * a.num_q_heads + h) * D +
+                                              half * (D / 2));
+        for (int q4 = 0; q4 < D / 16; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else if (all_ok) {
       tc_fence_after();
       const float lrow = half_l[0][r] + half_l[1][r];
       const float inv_l = (row_valid && lrow > 0.0f) ? 1.0f / lrow : 0.0f;
@@ -540,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     if (tid == 0) {
-      a.visited[row_id] = n;
+      a.visited[row_id] = ncomp;
       a.skipped[row_id] = nskip;
       if (a.skipbits != nullptr)
         for (int t = n; t < a.kmax; ++t) a.skipbits[row_id * a.kmax + t] = 0;

@@ -226,6 +226,24 @@ COSA_API int cosa_attn_delta(const cosa_shape_t* shape, const void* q, const voi
                     uint8_t* skipbits, void* workspace, size_t ws_bytes, cosa_stream_t stream);
 
 /*
+ * OSK attention in logical-mask execution, for the ablation of §4.3
+ * "Physical jumping over pages": the kernel walks every entry of each row's
+ * list and computes only those with keep[h, I, t] != 0 (device uint8
+ * [Hq, NQB, kmax]); the others are passed over by each warp role with no
+ * copy, MMA or vote, as a block-sparse kernel with a mask would.  With the
+ * list 0, 1, ..., i of all causal blocks and keep marking the selected ones,
+ * this is the same computation as cosa_attn on the selected blocks in
+ * ascending order.  visited counts the computed entries; skipbits is indexed
+ * by list entry (0 where keep is 0).  A row with no kept entry is written as
+ * zeros.  keep must not be NULL; everything else as cosa_attn.
+ */
+COSA_API int cosa_attn_masked(const cosa_shape_t* shape, const void* q, const void* k_pages, const void* v_pages,
+                     const int32_t* page_table, const int32_t* order, const int32_t* count,
+                     int32_t kmax, const uint8_t* keep, float tau, void* out, int32_t* visited,
+                     int32_t* skipped, uint8_t* skipbits, void* workspace, size_t ws_bytes,
+                     cosa_stream_t stream);
+
+/*
  * Synchronise `stream`, read and clear the workspace's status word.
  * Returns COSA_OK, COSA_ERR_TIMEOUT, COSA_ERR_DEVICE or COSA_ERR_CUDA.
  */

@@ -122,3 +122,10 @@ def test_attn_rejects_tau_outside_unit_interval(lib):
         rc = lib.cosa_attn(ctypes.byref(sh), None, None, None, None, None, None, 52, ctypes.c_float(tau), None,
                            None, None, None, None, 0, None)
         assert rc == 1
+
+
+def test_attn_masked_needs_a_keep_mask(lib):
+    sh = _shape()
+    rc = lib.cosa_attn_masked(ctypes.byref(sh), None, None, None, None, None, None, 1024, None, ctypes.c_float(1e-4),
+                              None, None, None, None, None, 0, None)
+    assert rc == 1

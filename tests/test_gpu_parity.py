@@ -173,6 +173,33 @@ def test_attn_delta_matches_oracle_per_sequence(name, delta):
         assert int(res["skipped"].sum()) == 0
 
 
+@pytest.mark.parametrize("name,tau", [("ragged_b128_p64", 1e-3), ("qwen_mix", 1e-2), ("short_seqs", 1e-4)])
+def test_mask_loop_equals_physical_jump(name, tau):
+    """Logical-mask execution (every causal block walked, the unselected ones
+    passed over) computes exactly what the jump over the same blocks in
+    ascending order computes: same output bits, same counts."""
+    import bench
+    budget = 0.25
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], budget)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], budget, kmax, ws)
+    asc = bench.ascending_order(sel["order"])
+    jump = cosa.attn(d["batch"], d["q"], d["k_pages"], d["v_pages"], d["page_table"], asc, sel["count"], kmax, tau,
+                     ws)
+    cosa.check(ws)
+    o_full, c_full, keep, kmax_full = bench.masked_full_lists(sel["order"], sel["count"], w.seqlens, w.block_size)
+    ws_m, _ = cosa.alloc_workspace(d["batch"], 1.0)
+    mask = cosa.attn_masked(d["batch"], d["q"], d["k_pages"], d["v_pages"], d["page_table"], o_full, c_full,
+                            kmax_full, keep, tau, ws_m, skipbits=True)
+    cosa.check(ws_m)
+    assert torch.equal(mask["visited"], sel["count"])
+    assert torch.equal(mask["skipped"], jump["skipped"])
+    assert torch.equal(mask["out"], jump["out"])
+    # skip bits sit at list entries: exactly the kept entries can carry one
+    assert int((mask["skipbits"].int() * (1 - keep.int())).sum()) == 0
+    assert int(mask["skipbits"].int().sum()) == int(jump["skipped"].sum())
+
+
 def test_repeated_calls_are_deterministic():
     d = device("qwen_mix")
     ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
