@@ -20,7 +20,7 @@ import os
 import torch
 
 __all__ = [
-    "Batch", "CosaError", "alloc_workspace", "attn", "attn_delta", "attn_masked", "check", "lib", "proxy", "remap",
+    "Batch", "CosaError", "PAGES_HND", "PAGES_NHD", "alloc_workspace", "attn", "attn_delta", "attn_masked", "check", "lib", "proxy", "remap",
     "set_wait_limit", "tau_from_delta", "workspace_size", "LIB_PATH",
 ]
 
@@ -44,8 +44,12 @@ class _Shape(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("page_size", ctypes.c_int32),
         ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
         ("total_qblocks", ctypes.c_int32), ("max_seqlen", ctypes.c_int32),
-        ("cu_seqlens", ctypes.c_void_p), ("cu_qblocks", ctypes.c_void_p),
+        ("cu_seqlens", ctypes.c_void_p), ("cu_qblocks", ctypes.c_void_p), ("page_layout", ctypes.c_int32),
     ]
+
+
+PAGES_HND = 0   # k/v pages [P, Hkv, b_p, d]
+PAGES_NHD = 1   # k/v pages [P, b_p, Hkv, d]
 
 
 _P = ctypes.c_void_p
@@ -116,7 +120,7 @@ class Batch:
     """Shape of one packed prefill batch; owns device copies of cu_seqlens / cu_qblocks."""
 
     def __init__(self, seqlens, num_q_heads, num_kv_heads, head_dim, block_size, page_size, num_pages,
-                 max_pages_per_seq, device="cuda"):
+                 max_pages_per_seq, device="cuda", page_layout=PAGES_HND):
         self.seqlens = [int(x) for x in seqlens]
         b = int(block_size)
         qblocks = [(L + b - 1) // b for L in self.seqlens]
@@ -132,7 +136,8 @@ class Batch:
         self.total_tokens, self.total_qblocks = cu_s[-1], cu_q[-1]
         self.c = _Shape(len(self.seqlens), self.num_q_heads, self.num_kv_heads, self.head_dim, b, self.page_size,
                         int(num_pages), int(max_pages_per_seq), self.total_tokens, self.total_qblocks,
-                        max(self.seqlens), self.cu_seqlens.data_ptr(), self.cu_qblocks.data_ptr())
+                        max(self.seqlens), self.cu_seqlens.data_ptr(), self.cu_qblocks.data_ptr(),
+                        int(page_layout))
 
 
 def workspace_size(batch: Batch, budget: float):

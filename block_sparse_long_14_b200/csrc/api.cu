@@ -45,6 +45,7 @@ int check_shape(const cosa_shape_t* s) {
       s->total_qblocks < 1 || s->max_seqlen < 1 || s->max_pages_per_seq < 1)
     return COSA_ERR_INVALID_ARG;
   if (s->cu_seqlens == nullptr || s->cu_qblocks == nullptr) return COSA_ERR_INVALID_ARG;
+  if (s->page_layout != COSA_PAGES_HND && s->page_layout != COSA_PAGES_NHD) return COSA_ERR_INVALID_ARG;
   if (s->num_q_heads % s->num_kv_heads != 0) return COSA_ERR_INVALID_ARG;
   if (s->num_q_heads / s->num_kv_heads > 8) return COSA_ERR_UNSUPPORTED;
   if (s->head_dim != 64 && s->head_dim != 128) return COSA_ERR_UNSUPPORTED;
@@ -146,7 +147,7 @@ const char* cosa_error_string(int code) {
   }
 }
 
-int cosa_version(void) { return 100; }
+int cosa_version(void) { return 101; }
 
 void cosa_debug_set_wait_limit(uint32_t spins) { g_wait_limit.store(spins == 0 ? kDefaultWaitLimit : spins); }
 
@@ -199,6 +200,7 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   ka.max_pages_per_seq = shape->max_pages_per_seq;
   ka.num_pages = shape->num_pages;
   ka.nkb_total = shape->total_qblocks;
+  ka.nhd = shape->page_layout == COSA_PAGES_NHD ? 1 : 0;
   if (launch_kpool(ka, st) != cudaSuccess) return COSA_ERR_CUDA;
 
   ScoreArgs sa{};
@@ -293,13 +295,24 @@ int attn_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, con
     const cuuint32_t box[3] = {64, 1, 128};
     if (!make_map(&qmap, q, 3, dims, strides, box)) return COSA_ERR_CUDA;
   }
-  {
+  if (shape->page_layout == COSA_PAGES_HND) {
+    // rows of d elements, (page, kv head, token) major to minor
     const cuuint64_t rows = static_cast<cuuint64_t>(shape->num_pages) * shape->num_kv_heads * shape->page_size;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
     const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(shape->page_size)};
     if (!make_map(&kmap, k_pages, 2, dims, strides, box)) return COSA_ERR_CUDA;
     if (!make_map(&vmap, v_pages, 2, dims, strides, box)) return COSA_ERR_CUDA;
+  } else {
+    // (d, kv head, page * b_p + token): a box of one kv head's b_p tokens lands
+    // in shared memory exactly like the HND box
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(shape->num_kv_heads),
+                                static_cast<cuuint64_t>(shape->num_pages) * shape->page_size};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(shape->num_kv_heads) * D * 2};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(shape->page_size)};
+    if (!make_map(&kmap, k_pages, 3, dims, strides, box)) return COSA_ERR_CUDA;
+    if (!make_map(&vmap, v_pages, 3, dims, strides, box)) return COSA_ERR_CUDA;
   }
   OskArgs oa{};
   oa.page_table = page_table;
@@ -314,6 +327,7 @@ int attn_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, con
   oa.skipped = skipped;
   oa.skipbits = skipbits;
   oa.keep = keep;
+  oa.nhd = shape->page_layout == COSA_PAGES_NHD ? 1 : 0;
   oa.status = reinterpret_cast<Status*>(workspace);
   oa.batch = shape->batch;
   oa.num_q_heads = Hq;
@@ -445,6 +459,7 @@ extern "C" int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, cons
   ka.max_pages_per_seq = shape->max_pages_per_seq;
   ka.num_pages = shape->num_pages;
   ka.nkb_total = shape->total_qblocks;
+  ka.nhd = shape->page_layout == COSA_PAGES_NHD ? 1 : 0;
   if (launch_kpool(ka, st) != cudaSuccess) return COSA_ERR_CUDA;
 
   ScoreArgs sa{};

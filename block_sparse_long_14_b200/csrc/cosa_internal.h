@@ -22,6 +22,7 @@ struct KPoolArgs {
   float* ks;      // [Hkv, NKB]
   Status* status;
   int batch, num_kv_heads, head_dim, block_size, page_size, max_pages_per_seq, num_pages, nkb_total;
+  int nhd;             // pages are [P, b_p, Hkv, d] instead of [P, Hkv, b_p, d]
 };
 
 struct ScoreArgs {
@@ -64,6 +65,7 @@ struct OskArgs {
   int32_t* skipped;
   uint8_t* skipbits;
   const uint8_t* keep;  // nullable: list entry t is computed only where keep[row, t] != 0
+  int nhd;              // pages are [P, b_p, Hkv, d] instead of [P, Hkv, b_p, d]
   Status* status;
   int batch, num_q_heads, num_kv_heads, block_size, page_size, max_pages_per_seq, num_pages;
   int nqb_total, kmax;

@@ -63,12 +63,16 @@ __global__ void __launch_bounds__(256) kpool_kernel(KPoolArgs a) {
       continue;
     }
     const int n_here = min(a.page_size, L - tok);
+    // token t of the page: HND [P, Hkv, b_p, d] or NHD [P, b_p, Hkv, d]
     const __nv_bfloat16* base =
-        a.k_pages + (static_cast<long>(page) * a.num_kv_heads + g) * a.page_size * D + lane * DPL;
+        a.k_pages + lane * DPL +
+        (a.nhd ? static_cast<long>(page) * a.page_size * a.num_kv_heads * D + static_cast<long>(g) * D
+               : (static_cast<long>(page) * a.num_kv_heads + g) * a.page_size * D);
+    const long tstride = a.nhd ? static_cast<long>(a.num_kv_heads) * D : D;
 #pragma unroll 8
     for (int t = 0; t < n_here; ++t) {
       if constexpr (DPL == 4) {
-        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(base + static_cast<long>(t) * D));
+        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(base + static_cast<long>(t) * tstride));
         const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
         const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
         acc[0] = __fadd_rn(acc[0], __low2float(lo));
@@ -76,7 +80,7 @@ __global__ void __launch_bounds__(256) kpool_kernel(KPoolArgs a) {
         acc[2] = __fadd_rn(acc[2], __low2float(hi));
         acc[3] = __fadd_rn(acc[3], __high2float(hi));
       } else {
-        const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(base + static_cast<long>(t) * D));
+        const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(base + static_cast<long>(t) * tstride));
         const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&raw);
         acc[0] = __fadd_rn(acc[0], __low2float(v));
         acc[1] = __fadd_rn(acc[1], __high2float(v));

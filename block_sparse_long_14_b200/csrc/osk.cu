@@ -123,8 +123,9 @@ __device__ void manual_block_copy(unsigned char* stage, const __nv_bfloat16* poo
     if (row < nvalid) {
       const int page = __ldg(pt_row + j * ppb + row / a.page_size);
       if (page >= 0 && page < a.num_pages) {
-        const __nv_bfloat16* src =
-            pool + ((static_cast<long>(page) * a.num_kv_heads + g) * a.page_size + row % a.page_size) * D + ch * 8;
+        const long tok = a.nhd ? (static_cast<long>(page) * a.page_size + row % a.page_size) * a.num_kv_heads + g
+                               : (static_cast<long>(page) * a.num_kv_heads + g) * a.page_size + row % a.page_size;
+        const __nv_bfloat16* src = pool + tok * D + ch * 8;
         v = __ldg(reinterpret_cast<const uint4*>(src));
       } else {
         report(a.status, kErrBounds, 0x300);
@@ -273,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       // a bad page id sends the block down the checked path
       const bool pages_ok = __all_sync(0xffffffffu, lane >= ppb || (page >= 0 && page < a.num_pages));
       const bool via_tma = jvalid && nvalid == b && pages_ok;
-      const int row = (page * a.num_kv_heads + g) * a.page_size;  // lane u < ppb: first pool row of page u
+      // lane u < ppb: first pool row of page u (HND), or its token row (NHD, with kv head g as y)
+      const int row = a.nhd ? page * a.page_size : (page * a.num_kv_heads + g) * a.page_size;
       // look-ahead loads, consumed one and two blocks later
       const int pg_nn = page_of(j_nn);
       const int j_nnn = block_id(t + 3);
@@ -290,8 +292,11 @@ __global__ void __launch_bounds__(kThreads, 2)
           __syncwarp();
           if (lane < ppb) {
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_2d(stage + c * (BK * 128) + lane * a.page_size * 128, map, full, c * 64, row);
+            for (int c = 0; c < D / 64; ++c) {
+              unsigned char* dst = stage + c * (BK * 128) + lane * a.page_size * 128;
+              if (a.nhd) tma_load_3d(dst, map, full, c * 64, g, row);
+              else tma_load_2d(dst, map, full, c * 64, row);
+            }
           }
           __syncwarp();
         } else {

@@ -74,6 +74,9 @@ typedef enum cosa_status {
  *   max_seqlen         max L_s (sizes the per-row lists)
  *   cu_seqlens         device int32 [B+1]: token offset of each sequence in q/out
  *   cu_qblocks         device int32 [B+1]: q-block offset of each sequence
+ *   page_layout        COSA_PAGES_HND (k/v pages [P, Hkv, b_p, d]) or
+ *                      COSA_PAGES_NHD ([P, b_p, Hkv, d]); both read through
+ *                      the same page_table
  *
  * The host fields must agree with the device arrays; the kernels trust them
  * for grid sizes and check every derived index against them.
@@ -92,7 +95,12 @@ typedef struct cosa_shape {
   int32_t max_seqlen;
   const int32_t* cu_seqlens;
   const int32_t* cu_qblocks;
+  int32_t page_layout;   /* COSA_PAGES_HND or COSA_PAGES_NHD */
 } cosa_shape_t;
+
+/* Page pool layouts of k_pages / v_pages. */
+#define COSA_PAGES_HND 0   /* [P, Hkv, b_p, d]: a (page, kv head) tile is contiguous */
+#define COSA_PAGES_NHD 1   /* [P, b_p, Hkv, d]: a token's kv heads are contiguous (paged-attention engines) */
 
 /*
  * Workspace bytes needed by cosa_proxy / cosa_attn for `shape` at stage-1

@@ -129,3 +129,10 @@ def test_attn_masked_needs_a_keep_mask(lib):
     rc = lib.cosa_attn_masked(ctypes.byref(sh), None, None, None, None, None, None, 1024, None, ctypes.c_float(1e-4),
                               None, None, None, None, None, 0, None)
     assert rc == 1
+
+
+def test_page_layouts(lib):
+    assert _ws(_shape(page_layout=0), 0.1)[0] > 0
+    assert _ws(_shape(page_layout=1), 0.1)[0] > 0
+    assert _ws(_shape(page_layout=2), 0.1)[0] == 0
+    assert lib.cosa_version() >= 101

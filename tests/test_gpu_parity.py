@@ -200,6 +200,31 @@ def test_mask_loop_equals_physical_jump(name, tau):
     assert int(mask["skipbits"].int().sum()) == int(jump["skipped"].sum())
 
 
+@pytest.mark.parametrize("name", ["ragged_b128_p64", "ragged_b128_p16_g1", "d64_b128_p32", "b64_g8"])
+def test_nhd_pages_give_identical_results(name):
+    """The same pools stored [P, b_p, Hkv, d] (NHD) instead of [P, Hkv, b_p, d]:
+    identical lists, HRM flags, outputs and skip decisions."""
+    budget, tau = 0.25, 1e-3
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], budget)
+    sel = cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], budget, kmax, ws)
+    sel = {k: v.clone() for k, v in sel.items()}
+    res = gu.run_attn(d, sel, kmax, tau, ws)
+    kn = d["k_pages"].permute(0, 2, 1, 3).contiguous()
+    vn = d["v_pages"].permute(0, 2, 1, 3).contiguous()
+    bn = cosa.Batch(w.seqlens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.page_size, w.num_pages,
+                    w.max_pages_per_seq, page_layout=cosa.PAGES_NHD)
+    sel_n = cosa.proxy(bn, d["q"], kn, d["page_table"], budget, kmax, ws)
+    cosa.check(ws)
+    for k in sel:
+        assert torch.equal(sel_n[k], sel[k]), k
+    res_n = cosa.attn(bn, d["q"], kn, vn, d["page_table"], sel_n["order"], sel_n["count"], kmax, tau, ws,
+                      skipbits=True)
+    cosa.check(ws)
+    for k in ("out", "visited", "skipped", "skipbits"):
+        assert torch.equal(res_n[k], res[k]), k
+
+
 def test_repeated_calls_are_deterministic():
     d = device("qwen_mix")
     ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
