@@ -35,7 +35,7 @@ namespace cosa {
 static constexpr float kTiny = 1.17549435e-38f;  // 2^-126: smallest normal fp32
 
 // ============================================================================ kpool
-template <int D>
+template <int D, bool NHD>
 __global__ void __launch_bounds__(256) kpool_kernel(KPoolArgs a) {
   constexpr int DPL = D / 32;  // dims per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -66,9 +66,9 @@ __global__ void __launch_bounds__(256) kpool_kernel(KPoolArgs a) {
     // token t of the page: HND [P, Hkv, b_p, d] or NHD [P, b_p, Hkv, d]
     const __nv_bfloat16* base =
         a.k_pages + lane * DPL +
-        (a.nhd ? static_cast<long>(page) * a.page_size * a.num_kv_heads * D + static_cast<long>(g) * D
-               : (static_cast<long>(page) * a.num_kv_heads + g) * a.page_size * D);
-    const long tstride = a.nhd ? static_cast<long>(a.num_kv_heads) * D : D;
+        (NHD ? static_cast<long>(page) * a.page_size * a.num_kv_heads * D + static_cast<long>(g) * D
+             : (static_cast<long>(page) * a.num_kv_heads + g) * a.page_size * D);
+    const long tstride = NHD ? static_cast<long>(a.num_kv_heads) * D : D;
 #pragma unroll 8
     for (int t = 0; t < n_here; ++t) {
       if constexpr (DPL == 4) {
@@ -942,8 +942,13 @@ static cudaError_t launch_proxy_kernel(const ScoreArgs& a, int GT, cudaStream_t 
 cudaError_t launch_kpool(const KPoolArgs& a, cudaStream_t stream) {
   const long items = static_cast<long>(a.nkb_total) * a.num_kv_heads;
   const unsigned grid = static_cast<unsigned>((items + 7) / 8);
-  if (a.head_dim == 128) kpool_kernel<128><<<grid, 256, 0, stream>>>(a);
-  else kpool_kernel<64><<<grid, 256, 0, stream>>>(a);
+  if (a.nhd) {
+    if (a.head_dim == 128) kpool_kernel<128, true><<<grid, 256, 0, stream>>>(a);
+    else kpool_kernel<64, true><<<grid, 256, 0, stream>>>(a);
+  } else {
+    if (a.head_dim == 128) kpool_kernel<128, false><<<grid, 256, 0, stream>>>(a);
+    else kpool_kernel<64, false><<<grid, 256, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 
