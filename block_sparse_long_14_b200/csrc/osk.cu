@@ -68,17 +68,18 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[1];
-  uint64_t p_full[2];   // softmax verdict (and P, if kept) for block t, by t & 1
-  uint64_t o_done[2];   // P V of kept block c has completed, by c & 1
+  uint64_t s_full[1];   // S of the c-th computed block is in TMEM (phase c & 1)
+  uint64_t p_full[2];   // softmax verdict (and P, if kept) for the c-th computed block, by c & 1
+  uint64_t o_done[2];   // P V of the k-th kept block has completed, by k & 1
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort;
-  int skip_flag[2];
-  int vote[2][kSoftmaxWarps];
+  int skip_flag[2];            // by c & 1, like p_full
+  int vote[2][kSoftmaxWarps];  // by c & 1
   int vote_end[kSoftmaxWarps];
-  float half_max[2][2][kBQ];   // [t & 1][half][row]: exchange of half-row maxima;
-                               // the epilogue reuses slot [n & 1] for partial row sums
+  float half_max[2][2][kBQ];   // [c & 1][half][row]: exchange of half-row maxima; the
+                               // epilogue reuses the slot after the last computed block
+                               // for the partial row sums
 };
 
 template <int D, int BK>
