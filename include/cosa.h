@@ -122,7 +122,8 @@ COSA_API int cosa_workspace_init(void* workspace, size_t ws_bytes, cosa_stream_t
  * KAP proxy (§4.2, Appendix C.1): stage-1 selection and visit order.
  *
  *   q           device bf16 [T, Hq, d]
- *   k_pages     device bf16 [P, Hkv, b_p, d]  (one (page, kv head) tile contiguous)
+ *   k_pages     device bf16 [P, Hkv, b_p, d], or [P, b_p, Hkv, d] when
+ *               shape->page_layout is COSA_PAGES_NHD
  *   page_table  device int32 [B, max_pages_per_seq]; entry (s, p) is the
  *               physical page of tokens [p*b_p, (p+1)*b_p) of sequence s.
  *               Entries past the sequence's last page are not read.
@@ -145,7 +146,9 @@ COSA_API int cosa_workspace_init(void* workspace, size_t ws_bytes, cosa_stream_t
  *   HRM: key block j is HRM iff it is the argmax over j' <= i (lowest index
  *     on ties) of some valid sub-row's score;
  *   order: (HRM first, score descending, block index ascending), first k_i.
- * The workspace holds the pooled int8 keys between the two kernels.
+ * The workspace holds the pooled int8 keys and query vectors between the
+ * three kernels the call enqueues (key pooling, query pooling, scoring and
+ * selection).
  */
 COSA_API int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages,
                const int32_t* page_table, float budget, int32_t kmax,
