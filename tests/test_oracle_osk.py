@@ -137,6 +137,23 @@ def test_threshold_edges():
     assert osk.osk_tile(q, qpos, blocks, [1, 0], 0.999, scale)[1][0] == False  # noqa: E712
 
 
+def test_tau_at_or_above_one_follows_the_rule_as_written():
+    """tau = delta / L can exceed 1 for a sequence shorter than delta.  The rule
+    stays "skip iff delta < ln tau": a block whose logits sit 0.5 above the
+    running max is skipped at tau = 2 (ln 2 = 0.69) and kept at tau = 1.5
+    (ln 1.5 = 0.41); a skipped block changes neither m nor l nor O."""
+    q, qpos, blocks, scale, VA, VB = _two_block_tile(low=0.5)
+    out, skipped, delta = osk.osk_tile(q, qpos, blocks, [0, 1], 2.0, scale)
+    assert skipped.tolist() == [False, True]
+    assert delta[1] == pytest.approx(0.5)
+    assert np.abs(out - VA.mean(axis=0)[None, :]).max() < 1e-12
+    out, skipped, _ = osk.osk_tile(q, qpos, blocks, [0, 1], 1.5, scale)
+    assert skipped.tolist() == [False, False]
+    w_b = math.exp(0.5)
+    expect = (VA.sum(0) + w_b * VB.sum(0)) / (16 + 16 * w_b)
+    assert np.abs(out - expect[None, :]).max() < 1e-12
+
+
 @pytest.mark.parametrize("tau", [1e-4, 1e-3, 1e-2, 1e-1])
 def test_skip_error_bound(tau):
     """Each skipped key weighs < tau relative to the row max, and l >= 1, so
