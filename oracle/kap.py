@@ -29,6 +29,10 @@ follows the same definitions):
   * Budget: bp = floor(budget * 1e4 + 0.5); k_i = max(1, ceil(n_i bp / 1e4)).
   * Order key: (HRM first, score descending, block index ascending); keep the
     first k_i.  No block is forced in.
+  * Top-p (the pages' stage-1 rule, §5.1 "Hyperparameters"; the pages give
+    p only): block j's mass is n_tok(j) exp(z_j), z_j the mean logit
+    estimated from the pooled score; k_i is the shortest prefix of the
+    order above whose share of the row's mass reaches p (top_p_count).
 """
 
 from __future__ import annotations
@@ -213,6 +217,100 @@ def kap_proxy(q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, block_siz
         tok0 += L
         blk0 += nqb
     return dict(order=order, count=count, n_hrm=n_hrm, hrm=hrm_out, kmax=kmax)
+
+
+def top_p_count(ordered_scores: np.ndarray, ordered_ntok: np.ndarray, zscale: float, p: float,
+                eps: float = 1e-6):
+    """Stage-1 Top-p cut of one row (§5.1 "Hyperparameters", Appendix D.1: the
+    pages fix p, not the mass; this is the reading of this build).
+
+    ordered_scores: float32 [n_i] pooled scores of the candidates, already in
+    the visit order (HRM first, score descending, block index ascending);
+    ordered_ntok: their token counts; zscale > 0 turns a pooled score into the
+    mean logit between the q-block's rows and the block's keys:
+      z_j = score_j * zscale,  zscale = (M_q / 127) / (n_rows * sqrt(d)),
+    with M_q the q-block sum's quantisation scale (dropped from the ranking
+    score, needed for a mass).  Block j's share of the row's attention is
+      w_j = n_tok(j) exp(z_j - max z) / sum_j' n_tok(j') exp(z_j' - max z)
+    (fp64).  k = the shortest prefix of the order whose share is >= p (at
+    least 1); p = 1 keeps the whole list, as it does in exact arithmetic
+    even where a far tail's fp64 mass underflows to zero.  Also returned: the window
+    [k_lo, k_hi] of prefix lengths whose share lies within eps of p, where a
+    computation in another precision may legitimately cut instead.
+    Returns (k, k_lo, k_hi).
+    """
+    if not 0.0 < p <= 1.0:
+        raise ValueError("p must lie in (0, 1]")
+    z = ordered_scores.astype(np.float64) * float(zscale)
+    mass = ordered_ntok.astype(np.float64) * np.exp(z - z.max())
+    cum = np.cumsum(mass)
+    share = cum / cum[-1]
+    share[-1] = 1.0
+    n = share.shape[0]
+    if p >= 1.0:
+        return n, n, n            # every mass is positive: only the whole list reaches 1
+    k = int(np.searchsorted(share, p, side="left")) + 1     # first prefix with share >= p
+    k = min(max(k, 1), n)
+    near = np.nonzero(np.abs(share - p) <= eps)[0]
+    k_lo = min(k, int(near.min()) + 1) if near.size else k
+    k_hi = max(k, int(near.max()) + 2) if near.size else k
+    return k, k_lo, min(k_hi, n)
+
+
+def kap_proxy_top_p(q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, block_size, p: float,
+                    g: int = SUB_ROWS, eps: float = 1e-6):
+    """KAP with the Top-p stage-1 cut instead of a budget fraction.
+
+    Same scores, HRM flags and order as kap_proxy; each row keeps the
+    top_p_count prefix of its full flag-grouped order.  Returns dict with
+    order int32 [Hq, NQB, kmax] (kmax = the longest sequence's q-blocks,
+    -1 pad), count, count_lo, count_hi int32 [Hq, NQB] (the cut and its
+    eps window), n_hrm, hrm.
+    """
+    Hq = q_bits.shape[1]
+    G = Hq // num_kv_heads
+    b = block_size
+    d = q_bits.shape[2]
+    nqbs = [(L + b - 1) // b for L in seqlens]
+    NQB = int(sum(nqbs))
+    kmax = max(nqbs)
+    order = np.full((Hq, NQB, kmax), -1, dtype=np.int32)
+    hrm_out = np.zeros((Hq, NQB, kmax), dtype=np.uint8)
+    count = np.zeros((Hq, NQB), dtype=np.int32)
+    count_lo = np.zeros((Hq, NQB), dtype=np.int32)
+    count_hi = np.zeros((Hq, NQB), dtype=np.int32)
+    n_hrm = np.zeros((Hq, NQB), dtype=np.int32)
+    tok0, blk0 = 0, 0
+    for s, L in enumerate(seqlens):
+        nqb = nqbs[s]
+        kf = f32(gather_tokens(k_pages_bits, page_table[s], L))
+        ksum, ntok = pool_keys(kf, L, b)
+        k8, ks = quantize_keys(ksum, ntok)
+        qf = f32(q_bits[tok0:tok0 + L])
+        sub, blk, sub_valid = pool_queries(qf, L, b, g)
+        q8_sub, _ = quantize_int8(sub)
+        q8_blk, Mq = quantize_int8(blk)              # Mq [nqb, Hq]
+        R = sub.shape[1]
+        nrows = np.array([min(b, L - i * b) for i in range(nqb)], dtype=np.float64)
+        for h in range(Hq):
+            kv = h // G
+            s_blk = scores_from_dots(int_dots(q8_blk[:, h], k8[:, kv]), ks[:, kv])
+            s_sub = scores_from_dots(int_dots(q8_sub[:, :, h].reshape(nqb * R, -1), k8[:, kv]),
+                                     ks[:, kv]).reshape(nqb, R, nqb)
+            for i in range(nqb):
+                n_i = i + 1
+                o, fl, _ = select_row(s_blk[i, :n_i], s_sub[i, :, :n_i], sub_valid[i], n_i)
+                zscale = (float(Mq[i, h]) / 127.0) / (nrows[i] * math.sqrt(d))
+                k, k_lo, k_hi = top_p_count(s_blk[i, o], ntok[o], zscale, p, eps)
+                I = blk0 + i
+                order[h, I, :k] = o[:k]
+                hrm_out[h, I, :k] = fl[:k]
+                count[h, I], count_lo[h, I], count_hi[h, I] = k, k_lo, k_hi
+                n_hrm[h, I] = int(fl[:k].sum())
+        tok0 += L
+        blk0 += nqb
+    return dict(order=order, count=count, count_lo=count_lo, count_hi=count_hi, n_hrm=n_hrm, hrm=hrm_out,
+                kmax=kmax)
 
 
 def remap(order, count, page_table, seqlens, block_size, page_size):
