@@ -22,6 +22,9 @@ open points fixed as stated in each function.
   dense    -- brute-force dense causal softmax attention, fp64 (§3.1), used as
               the closed form the OSK oracle must reduce to at budget 100% and
               tau = 0.
+  _layout  -- which q-blocks exist and where their rows sit in the packed Q,
+              for full prefill and for prefill after a cached prefix
+              (q_len < kv_len; a reading, the pages treat full prefill only).
 
 Parity status: the proxy's score and HRM definitions are this oracle's own
 reading of the empty "Block ranking" paragraph (§4.2); they are pinned by

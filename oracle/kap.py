@@ -42,6 +42,7 @@ import math
 import numpy as np
 
 from ._bf16 import f32, gather_tokens
+from ._layout import num_query_blocks, query_blocks
 
 SUB_ROWS = 16          # g: query rows per HRM sub-row
 _F127 = np.float32(127.0)
@@ -107,12 +108,14 @@ def quantize_keys(sums: np.ndarray, ntok: np.ndarray):
     return k8, ks
 
 
-def pool_queries(qf: np.ndarray, length: int, b: int, g: int = SUB_ROWS):
+def pool_queries(qf: np.ndarray, length: int, b: int, g: int = SUB_ROWS, offset: int = 0):
     """Per q-block: the fp32 sums of its R = b/g sub-rows and of the whole block.
 
-    qf: float32 [length, Hq, d].  A sub-row sums its valid rows one by one; a
-    sub-row with no valid row sums to +0.  The block sum folds the R sub-row
-    sums in order starting from +0.
+    qf: float32 [length, Hq, d] by absolute position; the rows at positions
+    below `offset` (a cached prefix) are absent and never read.  A row is
+    valid iff offset <= position < length.  A sub-row sums its valid rows one
+    by one; a sub-row with no valid row sums to +0 and is invalid.  The block
+    sum folds the R sub-row sums in order starting from +0.
     Returns (sub float32 [nqb, R, Hq, d], blk float32 [nqb, Hq, d],
              sub_valid bool [nqb, R]).
     """
@@ -125,12 +128,12 @@ def pool_queries(qf: np.ndarray, length: int, b: int, g: int = SUB_ROWS):
     first_row = (np.arange(nqb)[:, None] * b + np.arange(R)[None, :] * g)   # [nqb, R]
     sub = np.zeros((nqb, R, H, d), dtype=np.float32)
     for t in range(g):
-        valid = (first_row + t) < length
+        valid = ((first_row + t) < length) & ((first_row + t) >= offset)
         sub[valid] = (sub[valid] + rows[:, :, t][valid]).astype(np.float32)
     blk = np.zeros((nqb, H, d), dtype=np.float32)
     for r in range(R):
         blk = (blk + sub[:, r]).astype(np.float32)
-    return sub, blk, first_row < length
+    return sub, blk, (first_row < length) & (first_row + g > offset)
 
 
 def int_dots(a8: np.ndarray, b8: np.ndarray) -> np.ndarray:
@@ -166,56 +169,72 @@ def select_row(score: np.ndarray, sub_scores: np.ndarray, sub_valid: np.ndarray,
     return order, hrm[order], hrm
 
 
-def kap_proxy(q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, block_size, budget,
-              g: int = SUB_ROWS, kmax: int | None = None, heads=None):
-    """KAP over a packed batch.
+def _scored_rows(q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, block_size, g,
+                 heads, q_lens):
+    """Every (query head h, list row I) of a packed batch with what its selection needs.
 
-    Returns dict with order int32 [Hq, NQB, kmax] (-1 pad), count int32
-    [Hq, NQB], n_hrm int32 [Hq, NQB], hrm uint8 [Hq, NQB, kmax], kmax, and
-    for inspection the per-sequence block scores.
-    `heads` restricts the work to a subset of query heads (others stay -1/0).
+    Yields (h, I, i, s_blk [n_i], s_sub [R, n_i], sub_valid [R], ntok [n_i],
+    M_q, n_rows): block and sub-row scores over the candidates j = 0..i, the
+    key blocks' token counts, the q-block sum's max-abs and its number of
+    query rows.  q_lens as in oracle._layout.query_blocks.
     """
     Hq = q_bits.shape[1]
-    Hkv = num_kv_heads
-    G = Hq // Hkv
+    G = Hq // num_kv_heads
     b = block_size
-    bp = budget_bp(budget)
-    nqbs = [(L + b - 1) // b for L in seqlens]
-    NQB = int(sum(nqbs))
-    if kmax is None:
-        kmax = keep_count(max(nqbs), bp)
-    order = np.full((Hq, NQB, kmax), -1, dtype=np.int32)
-    hrm_out = np.zeros((Hq, NQB, kmax), dtype=np.uint8)
-    count = np.zeros((Hq, NQB), dtype=np.int32)
-    n_hrm = np.zeros((Hq, NQB), dtype=np.int32)
     heads = range(Hq) if heads is None else heads
-    tok0, blk0 = 0, 0
-    for s, L in enumerate(seqlens):
-        nqb = nqbs[s]
+    I0 = 0
+    for s, (off, i0, nqb, tq0) in enumerate(query_blocks(seqlens, q_lens, b)):
+        L = int(seqlens[s])
         kf = f32(gather_tokens(k_pages_bits, page_table[s], L))
         ksum, ntok = pool_keys(kf, L, b)
         k8, ks = quantize_keys(ksum, ntok)
-        qf = f32(q_bits[tok0:tok0 + L])
-        sub, blk, sub_valid = pool_queries(qf, L, b, g)
+        qf = np.zeros((L,) + q_bits.shape[1:], dtype=np.float32)
+        qf[off:] = f32(q_bits[tq0:tq0 + L - off])      # query t at position off + t
+        sub, blk, sub_valid = pool_queries(qf, L, b, g, off)
         q8_sub, _ = quantize_int8(sub)     # [nqb, R, Hq, d]
-        q8_blk, _ = quantize_int8(blk)     # [nqb, Hq, d]
+        q8_blk, Mq = quantize_int8(blk)    # [nqb, Hq, d], [nqb, Hq]
         R = sub.shape[1]
         for h in heads:
             kv = h // G
             s_blk = scores_from_dots(int_dots(q8_blk[:, h], k8[:, kv]), ks[:, kv])       # [nqb, nkb]
             s_sub = scores_from_dots(int_dots(q8_sub[:, :, h].reshape(nqb * R, -1), k8[:, kv]),
                                      ks[:, kv]).reshape(nqb, R, nqb)
-            for i in range(nqb):
-                n_i = i + 1
-                k_i = keep_count(n_i, bp)
-                o, fl, _ = select_row(s_blk[i, :n_i], s_sub[i, :, :n_i], sub_valid[i], k_i)
-                I = blk0 + i
-                order[h, I, :k_i] = o
-                hrm_out[h, I, :k_i] = fl
-                count[h, I] = k_i
-                n_hrm[h, I] = int(fl.sum())
-        tok0 += L
-        blk0 += nqb
+            for i in range(i0, nqb):
+                n_rows = min(L, (i + 1) * b) - max(off, i * b)
+                yield (h, I0 + i - i0, i, s_blk[i, :i + 1], s_sub[i, :, :i + 1], sub_valid[i],
+                       ntok[:i + 1], float(Mq[i, h]), n_rows)
+        I0 += nqb - i0
+
+
+def kap_proxy(q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, block_size, budget,
+              g: int = SUB_ROWS, kmax: int | None = None, heads=None, q_lens=None):
+    """KAP over a packed batch.
+
+    q_lens: per-sequence query counts for prefill after a cached prefix
+    (default: every token is a query); q_bits then holds only those rows.
+    Returns dict with order int32 [Hq, NQB, kmax] (-1 pad; NQB = the present
+    q-blocks), count int32 [Hq, NQB], n_hrm int32 [Hq, NQB], hrm uint8
+    [Hq, NQB, kmax], kmax.
+    `heads` restricts the work to a subset of query heads (others stay -1/0).
+    """
+    Hq = q_bits.shape[1]
+    b = block_size
+    bp = budget_bp(budget)
+    NQB = num_query_blocks(seqlens, q_lens, b)
+    if kmax is None:
+        kmax = keep_count(max((L + b - 1) // b for L in seqlens), bp)
+    order = np.full((Hq, NQB, kmax), -1, dtype=np.int32)
+    hrm_out = np.zeros((Hq, NQB, kmax), dtype=np.uint8)
+    count = np.zeros((Hq, NQB), dtype=np.int32)
+    n_hrm = np.zeros((Hq, NQB), dtype=np.int32)
+    for h, I, i, s_blk, s_sub, sub_valid, _, _, _ in _scored_rows(
+            q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, b, g, heads, q_lens):
+        k_i = keep_count(i + 1, bp)
+        o, fl, _ = select_row(s_blk, s_sub, sub_valid, k_i)
+        order[h, I, :k_i] = o
+        hrm_out[h, I, :k_i] = fl
+        count[h, I] = k_i
+        n_hrm[h, I] = int(fl.sum())
     return dict(order=order, count=count, n_hrm=n_hrm, hrm=hrm_out, kmax=kmax)
 
 
@@ -258,62 +277,40 @@ def top_p_count(ordered_scores: np.ndarray, ordered_ntok: np.ndarray, zscale: fl
 
 
 def kap_proxy_top_p(q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, block_size, p: float,
-                    g: int = SUB_ROWS, eps: float = 1e-6):
+                    g: int = SUB_ROWS, eps: float = 1e-6, q_lens=None):
     """KAP with the Top-p stage-1 cut instead of a budget fraction.
 
     Same scores, HRM flags and order as kap_proxy; each row keeps the
-    top_p_count prefix of its full flag-grouped order.  Returns dict with
-    order int32 [Hq, NQB, kmax] (kmax = the longest sequence's q-blocks,
-    -1 pad), count, count_lo, count_hi int32 [Hq, NQB] (the cut and its
-    eps window), n_hrm, hrm.
+    top_p_count prefix of its full flag-grouped order, with
+    zscale = (M_q / 127) / (n_rows sqrt(d)).  Returns dict with order int32
+    [Hq, NQB, kmax] (kmax = the longest sequence's block count, -1 pad),
+    count, count_lo, count_hi int32 [Hq, NQB] (the cut and its eps window),
+    n_hrm, hrm.
     """
-    Hq = q_bits.shape[1]
-    G = Hq // num_kv_heads
+    Hq, d = q_bits.shape[1], q_bits.shape[2]
     b = block_size
-    d = q_bits.shape[2]
-    nqbs = [(L + b - 1) // b for L in seqlens]
-    NQB = int(sum(nqbs))
-    kmax = max(nqbs)
+    NQB = num_query_blocks(seqlens, q_lens, b)
+    kmax = max((L + b - 1) // b for L in seqlens)
     order = np.full((Hq, NQB, kmax), -1, dtype=np.int32)
     hrm_out = np.zeros((Hq, NQB, kmax), dtype=np.uint8)
     count = np.zeros((Hq, NQB), dtype=np.int32)
     count_lo = np.zeros((Hq, NQB), dtype=np.int32)
     count_hi = np.zeros((Hq, NQB), dtype=np.int32)
     n_hrm = np.zeros((Hq, NQB), dtype=np.int32)
-    tok0, blk0 = 0, 0
-    for s, L in enumerate(seqlens):
-        nqb = nqbs[s]
-        kf = f32(gather_tokens(k_pages_bits, page_table[s], L))
-        ksum, ntok = pool_keys(kf, L, b)
-        k8, ks = quantize_keys(ksum, ntok)
-        qf = f32(q_bits[tok0:tok0 + L])
-        sub, blk, sub_valid = pool_queries(qf, L, b, g)
-        q8_sub, _ = quantize_int8(sub)
-        q8_blk, Mq = quantize_int8(blk)              # Mq [nqb, Hq]
-        R = sub.shape[1]
-        nrows = np.array([min(b, L - i * b) for i in range(nqb)], dtype=np.float64)
-        for h in range(Hq):
-            kv = h // G
-            s_blk = scores_from_dots(int_dots(q8_blk[:, h], k8[:, kv]), ks[:, kv])
-            s_sub = scores_from_dots(int_dots(q8_sub[:, :, h].reshape(nqb * R, -1), k8[:, kv]),
-                                     ks[:, kv]).reshape(nqb, R, nqb)
-            for i in range(nqb):
-                n_i = i + 1
-                o, fl, _ = select_row(s_blk[i, :n_i], s_sub[i, :, :n_i], sub_valid[i], n_i)
-                zscale = (float(Mq[i, h]) / 127.0) / (nrows[i] * math.sqrt(d))
-                k, k_lo, k_hi = top_p_count(s_blk[i, o], ntok[o], zscale, p, eps)
-                I = blk0 + i
-                order[h, I, :k] = o[:k]
-                hrm_out[h, I, :k] = fl[:k]
-                count[h, I], count_lo[h, I], count_hi[h, I] = k, k_lo, k_hi
-                n_hrm[h, I] = int(fl[:k].sum())
-        tok0 += L
-        blk0 += nqb
+    for h, I, i, s_blk, s_sub, sub_valid, ntok, Mq, n_rows in _scored_rows(
+            q_bits, k_pages_bits, page_table, seqlens, num_kv_heads, b, g, None, q_lens):
+        o, fl, _ = select_row(s_blk, s_sub, sub_valid, i + 1)
+        zscale = (Mq / 127.0) / (n_rows * math.sqrt(d))
+        k, k_lo, k_hi = top_p_count(s_blk[o], ntok[o], zscale, p, eps)
+        order[h, I, :k] = o[:k]
+        hrm_out[h, I, :k] = fl[:k]
+        count[h, I], count_lo[h, I], count_hi[h, I] = k, k_lo, k_hi
+        n_hrm[h, I] = int(fl[:k].sum())
     return dict(order=order, count=count, count_lo=count_lo, count_hi=count_hi, n_hrm=n_hrm, hrm=hrm_out,
                 kmax=kmax)
 
 
-def remap(order, count, page_table, seqlens, block_size, page_size):
+def remap(order, count, page_table, seqlens, block_size, page_size, q_lens=None):
     """Ordered key blocks -> physical pages, page by page (§4.3 "Any-order page visiting").
 
     pages[h, I, t * ppb + u] = page_table[s, order[h, I, t] * ppb + u] when
@@ -325,8 +322,9 @@ def remap(order, count, page_table, seqlens, block_size, page_size):
     out = np.full((Hq, NQB, kmax * ppb), -1, dtype=np.int32)
     t = np.arange(kmax)
     blk0 = 0
-    for s, L in enumerate(seqlens):
-        nqb = (L + block_size - 1) // block_size
+    for s, (_, i0, nb, _) in enumerate(query_blocks(seqlens, q_lens, block_size)):
+        L = int(seqlens[s])
+        nqb = nb - i0                                               # this sequence's list rows
         o = order[:, blk0:blk0 + nqb, :].astype(np.int64)            # [Hq, nqb, kmax]
         listed = t[None, None, :] < count[:, blk0:blk0 + nqb, None]
         for u in range(ppb):

@@ -31,6 +31,7 @@ import math
 import numpy as np
 
 from ._bf16 import f32, gather_tokens
+from ._layout import query_blocks
 
 
 def osk_tile(qrows, qpos, blocks, order, tau, scale):
@@ -88,28 +89,33 @@ class PagedSequence:
 
 
 def osk(q_bits, k_pages_bits, v_pages_bits, page_table, seqlens, num_kv_heads, block_size,
-        order, count, tau, units=None):
+        order, count, tau, units=None, q_lens=None):
     """OSK over a packed batch.
 
     order/count: the proxy's ordered lists [Hq, NQB, kmax] / [Hq, NQB].
+    q_lens: per-sequence query counts for prefill after a cached prefix
+    (default: every token is a query); query t of sequence s sits at
+    position L_s - Lq_s + t, and a tile holds the q-block's present rows.
+    tau: one threshold, or a sequence of one per sequence.
     units: optional iterable of (h, I) tiles to compute (default: all).
-    Returns dict: out fp64 [T, Hq, d] (NaN where not computed), visited and
+    Returns dict: out fp64 [Tq, Hq, d] (NaN where not computed), visited and
     skipped int32 [Hq, NQB] (-1 where not computed), skip bool and delta
     fp64 [Hq, NQB, kmax] (padding False / NaN).
     """
-    T, Hq, d = q_bits.shape
+    Tq, Hq, d = q_bits.shape
     G = Hq // num_kv_heads
     b = block_size
     scale = 1.0 / math.sqrt(d)
     kmax = order.shape[2]
     NQB = order.shape[1]
-    seq_of = np.concatenate([np.full((L + b - 1) // b, s) for s, L in enumerate(seqlens)])
-    blk0 = np.concatenate([[0], np.cumsum([(L + b - 1) // b for L in seqlens])])
-    tok0 = np.concatenate([[0], np.cumsum(seqlens)])
+    layout = query_blocks(seqlens, q_lens, b)
+    taus = list(tau) if np.ndim(tau) else [tau] * len(seqlens)
+    seq_of = np.concatenate([np.full(nb - i0, s) for s, (_, i0, nb, _) in enumerate(layout)])
+    blk0 = np.concatenate([[0], np.cumsum([nb - i0 for _, i0, nb, _ in layout])])
     if units is None:
         units = [(h, I) for h in range(Hq) for I in range(NQB)]
     units = sorted(set((int(h), int(I)) for h, I in units), key=lambda u: (seq_of[u[1]], u))
-    out = np.full((T, Hq, d), np.nan)
+    out = np.full((Tq, Hq, d), np.nan)
     visited = np.full((Hq, NQB), -1, dtype=np.int32)
     skipped = np.full((Hq, NQB), -1, dtype=np.int32)
     skip = np.zeros((Hq, NQB, kmax), dtype=bool)
@@ -121,14 +127,16 @@ def osk(q_bits, k_pages_bits, v_pages_bits, page_table, seqlens, num_kv_heads, b
             cache.clear()
             cache[s] = PagedSequence(k_pages_bits, v_pages_bits, page_table[s], seqlens[s], b)
         seq = cache[s]
-        i = I - blk0[s]
+        off, i0, _, tq0 = layout[s]
+        i = i0 + I - blk0[s]
         L = seqlens[s]
-        r0, r1 = i * b, min(L, (i + 1) * b)
-        qrows = f32(q_bits[tok0[s] + r0:tok0[s] + r1, h]).astype(np.float64)
+        r0, r1 = max(off, i * b), min(L, (i + 1) * b)        # absolute positions of the rows
+        rows = slice(tq0 + r0 - off, tq0 + r1 - off)          # their place in the packed Q
+        qrows = f32(q_bits[rows, h]).astype(np.float64)
         k_i = int(count[h, I])
         o, sk, de = osk_tile(qrows, np.arange(r0, r1), seq.block(h // G), order[h, I, :k_i],
-                             tau, scale)
-        out[tok0[s] + r0:tok0[s] + r1, h] = o
+                             taus[s], scale)
+        out[rows, h] = o
         visited[h, I] = k_i
         skipped[h, I] = int(sk.sum())
         skip[h, I, :k_i] = sk
