@@ -45,6 +45,7 @@ class _Shape(ctypes.Structure):
         ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
         ("total_qblocks", ctypes.c_int32), ("max_seqlen", ctypes.c_int32),
         ("cu_seqlens", ctypes.c_void_p), ("cu_qblocks", ctypes.c_void_p), ("page_layout", ctypes.c_int32),
+        ("kv_lens", ctypes.c_void_p), ("cu_kblocks", ctypes.c_void_p), ("total_kblocks", ctypes.c_int32),
     ]
 
 
@@ -117,27 +118,44 @@ def _check(rc, what):
 
 
 class Batch:
-    """Shape of one packed prefill batch; owns device copies of cu_seqlens / cu_qblocks."""
+    """Shape of one packed prefill batch; owns the device offset arrays.
+
+    seqlens: tokens per sequence (keys).  q_lens: optional queries per
+    sequence for prefill after a cached prefix; query t of sequence s is
+    token seqlens[s] - q_lens[s] + t, and q/out hold only the query rows.
+    Default: every token is a query.
+    """
 
     def __init__(self, seqlens, num_q_heads, num_kv_heads, head_dim, block_size, page_size, num_pages,
-                 max_pages_per_seq, device="cuda", page_layout=PAGES_HND):
+                 max_pages_per_seq, device="cuda", page_layout=PAGES_HND, q_lens=None):
         self.seqlens = [int(x) for x in seqlens]
+        self.q_lens = list(self.seqlens) if q_lens is None else [int(x) for x in q_lens]
+        if len(self.q_lens) != len(self.seqlens):
+            raise ValueError("q_lens and seqlens differ in length")
+        if any(not 1 <= Lq <= L for L, Lq in zip(self.seqlens, self.q_lens)):
+            raise ValueError("need 1 <= q_len <= seqlen for every sequence")
         b = int(block_size)
-        qblocks = [(L + b - 1) // b for L in self.seqlens]
-        cu_s = [0]
-        cu_q = [0]
-        for L, n in zip(self.seqlens, qblocks):
-            cu_s.append(cu_s[-1] + L)
-            cu_q.append(cu_q[-1] + n)
+        cu_s, cu_q, cu_k = [0], [0], [0]
+        for L, Lq in zip(self.seqlens, self.q_lens):
+            nkb = (L + b - 1) // b
+            cu_s.append(cu_s[-1] + Lq)
+            cu_q.append(cu_q[-1] + nkb - (L - Lq) // b)    # q-blocks that hold a query row
+            cu_k.append(cu_k[-1] + nkb)
         self.cu_seqlens = torch.tensor(cu_s, dtype=torch.int32, device=device)
         self.cu_qblocks = torch.tensor(cu_q, dtype=torch.int32, device=device)
+        self.prefix = q_lens is not None
+        self.kv_lens = torch.tensor(self.seqlens, dtype=torch.int32, device=device) if self.prefix else None
+        self.cu_kblocks = torch.tensor(cu_k, dtype=torch.int32, device=device) if self.prefix else None
         self.num_q_heads, self.num_kv_heads, self.head_dim = int(num_q_heads), int(num_kv_heads), int(head_dim)
         self.block_size, self.page_size = b, int(page_size)
-        self.total_tokens, self.total_qblocks = cu_s[-1], cu_q[-1]
+        self.total_tokens, self.total_qblocks, self.total_kblocks = cu_s[-1], cu_q[-1], cu_k[-1]
         self.c = _Shape(len(self.seqlens), self.num_q_heads, self.num_kv_heads, self.head_dim, b, self.page_size,
                         int(num_pages), int(max_pages_per_seq), self.total_tokens, self.total_qblocks,
                         max(self.seqlens), self.cu_seqlens.data_ptr(), self.cu_qblocks.data_ptr(),
-                        int(page_layout))
+                        int(page_layout),
+                        self.kv_lens.data_ptr() if self.prefix else None,
+                        self.cu_kblocks.data_ptr() if self.prefix else None,
+                        self.total_kblocks if self.prefix else 0)
 
 
 def workspace_size(batch: Batch, budget: float):

@@ -52,8 +52,15 @@ int check_shape(const cosa_shape_t* s) {
   if (s->block_size != 64 && s->block_size != 128) return COSA_ERR_UNSUPPORTED;
   if (s->page_size < 8 || s->page_size % 8 != 0 || s->block_size % s->page_size != 0) return COSA_ERR_UNSUPPORTED;
   if (s->max_pages_per_seq < ceil_div(s->max_seqlen, s->page_size)) return COSA_ERR_INVALID_ARG;
-  if (s->total_qblocks < ceil_div(s->max_seqlen, s->block_size)) return COSA_ERR_INVALID_ARG;
-  if (s->max_seqlen > s->total_tokens) return COSA_ERR_INVALID_ARG;
+  if (s->kv_lens == nullptr && s->total_qblocks < ceil_div(s->max_seqlen, s->block_size)) return COSA_ERR_INVALID_ARG;
+  if (s->kv_lens == nullptr) {
+    if (s->max_seqlen > s->total_tokens) return COSA_ERR_INVALID_ARG;
+  } else {
+    // prefill after a cached prefix: keys counted apart from the queries
+    if (s->cu_kblocks == nullptr || s->total_kblocks < 1) return COSA_ERR_INVALID_ARG;
+    if (s->total_kblocks < ceil_div(s->max_seqlen, s->block_size)) return COSA_ERR_INVALID_ARG;
+    if (s->total_kblocks < s->total_qblocks) return COSA_ERR_INVALID_ARG;
+  }
   // TMA row coordinates of the page pool are int32
   if (static_cast<long>(s->num_pages) * s->num_kv_heads * s->page_size >= (1L << 31)) return COSA_ERR_UNSUPPORTED;
   const int npow2 = next_pow2(ceil_div(s->max_seqlen, s->block_size));
@@ -64,8 +71,13 @@ int check_shape(const cosa_shape_t* s) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Workspace: status block, pooled int8 keys [Hkv, NQB, d], key scales
-// [Hkv, NQB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d].
+// Key blocks of the batch and their per-sequence offsets: the q-blocks'
+// unless a cached prefix separates them.
+int total_kblocks(const cosa_shape_t& s) { return s.kv_lens != nullptr ? s.total_kblocks : s.total_qblocks; }
+const int32_t* cu_kblocks(const cosa_shape_t& s) { return s.kv_lens != nullptr ? s.cu_kblocks : s.cu_qblocks; }
+
+// Workspace: status block, pooled int8 keys [Hkv, NKB, d], key scales
+// [Hkv, NKB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d].
 struct WsLayout {
   size_t kq_off, ks_off, qa_off, total;
 };
@@ -73,9 +85,9 @@ struct WsLayout {
 WsLayout ws_layout(const cosa_shape_t& s) {
   WsLayout w{};
   w.kq_off = kStatusBytes;
-  const size_t kq_bytes = static_cast<size_t>(s.num_kv_heads) * s.total_qblocks * s.head_dim;
+  const size_t kq_bytes = static_cast<size_t>(s.num_kv_heads) * total_kblocks(s) * s.head_dim;
   w.ks_off = align_up(w.kq_off + kq_bytes, 256);
-  w.qa_off = align_up(w.ks_off + static_cast<size_t>(s.num_kv_heads) * s.total_qblocks * 4, 256);
+  w.qa_off = align_up(w.ks_off + static_cast<size_t>(s.num_kv_heads) * total_kblocks(s) * 4, 256);
   const size_t qa_bytes =
       static_cast<size_t>(s.num_q_heads) * s.total_qblocks * (s.block_size / 16 + 1) * s.head_dim;
   w.total = align_up(w.qa_off + qa_bytes, 256);
@@ -147,7 +159,7 @@ const char* cosa_error_string(int code) {
   }
 }
 
-int cosa_version(void) { return 101; }
+int cosa_version(void) { return 102; }
 
 void cosa_debug_set_wait_limit(uint32_t spins) { g_wait_limit.store(spins == 0 ? kDefaultWaitLimit : spins); }
 
@@ -188,7 +200,8 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   ka.k_pages = static_cast<const __nv_bfloat16*>(k_pages);
   ka.page_table = page_table;
   ka.cu_seqlens = shape->cu_seqlens;
-  ka.cu_qblocks = shape->cu_qblocks;
+  ka.kv_lens = shape->kv_lens;
+  ka.cu_kblocks = cu_kblocks(*shape);
   ka.kq = reinterpret_cast<int8_t*>(ws + w.kq_off);
   ka.ks = reinterpret_cast<float*>(ws + w.ks_off);
   ka.status = status;
@@ -199,7 +212,7 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   ka.page_size = shape->page_size;
   ka.max_pages_per_seq = shape->max_pages_per_seq;
   ka.num_pages = shape->num_pages;
-  ka.nkb_total = shape->total_qblocks;
+  ka.nkb_total = total_kblocks(*shape);
   ka.nhd = shape->page_layout == COSA_PAGES_NHD ? 1 : 0;
   if (launch_kpool(ka, st) != cudaSuccess) return COSA_ERR_CUDA;
 
@@ -209,6 +222,8 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   sa.ks = ka.ks;
   sa.cu_seqlens = shape->cu_seqlens;
   sa.cu_qblocks = shape->cu_qblocks;
+  sa.kv_lens = shape->kv_lens;
+  sa.cu_kblocks = cu_kblocks(*shape);
   sa.order = order;
   sa.count = count;
   sa.n_hrm = n_hrm;
@@ -220,6 +235,7 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   sa.head_dim = shape->head_dim;
   sa.block_size = shape->block_size;
   sa.nqb_total = shape->total_qblocks;
+  sa.nkb_total = total_kblocks(*shape);
   sa.kmax = kmax;
   sa.bp = bp;
   sa.npow2_max = next_pow2(ceil_div(shape->max_seqlen, shape->block_size));
@@ -228,9 +244,9 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   sa.scratch_bytes = select_scratch_bytes(*shape, kmax, GT, sa.npow2_max);
   if (launch_qpool(sa, GT, st) != cudaSuccess) return COSA_ERR_CUDA;
   if (shape->head_dim == 128) {
-    // int8 key vectors as a [Hkv * NQB, 128] byte matrix for the tcgen05 score tiles
+    // int8 key vectors as a [Hkv * NKB, 128] byte matrix for the tcgen05 score tiles
     CUtensorMap kq_map;
-    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(shape->num_kv_heads) * shape->total_qblocks};
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(shape->num_kv_heads) * total_kblocks(*shape)};
     const cuuint64_t strides[1] = {128};
     const cuuint32_t box[2] = {128, 64};   // 64 key blocks x 128 int8 dims per score tile
     if (!make_map(&kq_map, sa.kq, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return COSA_ERR_CUDA;
@@ -253,6 +269,7 @@ int cosa_remap(const cosa_shape_t* shape, const int32_t* page_table, const int32
   ra.count = count;
   ra.cu_seqlens = shape->cu_seqlens;
   ra.cu_qblocks = shape->cu_qblocks;
+  ra.kv_lens = shape->kv_lens;
   ra.pages = pages;
   ra.status = nullptr;
   ra.batch = shape->batch;
@@ -320,6 +337,7 @@ int attn_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, con
   oa.count = count;
   oa.cu_seqlens = shape->cu_seqlens;
   oa.cu_qblocks = shape->cu_qblocks;
+  oa.kv_lens = shape->kv_lens;
   oa.k_pages = static_cast<const __nv_bfloat16*>(k_pages);
   oa.v_pages = static_cast<const __nv_bfloat16*>(v_pages);
   oa.out = static_cast<__nv_bfloat16*>(out);
@@ -433,9 +451,9 @@ extern "C" int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, cons
   if (!aligned16(q) || !aligned16(k_pages)) return COSA_ERR_INVALID_ARG;
   const int bp = budget_bp(budget);
   if (kmax < keep_count(ceil_div(shape->max_seqlen, shape->block_size), bp)) return COSA_ERR_INVALID_ARG;
-  // pooled keys [Hkv, NQB, d] int8, then scales [Hkv, NQB] fp32
-  const size_t kq_bytes = align_up(static_cast<size_t>(shape->num_kv_heads) * shape->total_qblocks * shape->head_dim, 256);
-  const size_t need = kq_bytes + static_cast<size_t>(shape->num_kv_heads) * shape->total_qblocks * 4;
+  // pooled keys [Hkv, NKB, d] int8, then scales [Hkv, NKB] fp32
+  const size_t kq_bytes = align_up(static_cast<size_t>(shape->num_kv_heads) * total_kblocks(*shape) * shape->head_dim, 256);
+  const size_t need = kq_bytes + static_cast<size_t>(shape->num_kv_heads) * total_kblocks(*shape) * 4;
   if (need > COSA_NOALLOC_SCRATCH_BYTES) return COSA_ERR_WORKSPACE;
   void* base = nullptr;
   rc = noalloc_scratch(&base);
@@ -447,7 +465,8 @@ extern "C" int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, cons
   ka.k_pages = static_cast<const __nv_bfloat16*>(k_pages);
   ka.page_table = page_table;
   ka.cu_seqlens = shape->cu_seqlens;
-  ka.cu_qblocks = shape->cu_qblocks;
+  ka.kv_lens = shape->kv_lens;
+  ka.cu_kblocks = cu_kblocks(*shape);
   ka.kq = reinterpret_cast<int8_t*>(scratch);
   ka.ks = reinterpret_cast<float*>(scratch + kq_bytes);
   ka.status = nullptr;
@@ -458,7 +477,7 @@ extern "C" int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, cons
   ka.page_size = shape->page_size;
   ka.max_pages_per_seq = shape->max_pages_per_seq;
   ka.num_pages = shape->num_pages;
-  ka.nkb_total = shape->total_qblocks;
+  ka.nkb_total = total_kblocks(*shape);
   ka.nhd = shape->page_layout == COSA_PAGES_NHD ? 1 : 0;
   if (launch_kpool(ka, st) != cudaSuccess) return COSA_ERR_CUDA;
 
@@ -468,6 +487,8 @@ extern "C" int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, cons
   sa.ks = ka.ks;
   sa.cu_seqlens = shape->cu_seqlens;
   sa.cu_qblocks = shape->cu_qblocks;
+  sa.kv_lens = shape->kv_lens;
+  sa.cu_kblocks = cu_kblocks(*shape);
   sa.order = order;
   sa.count = count;
   sa.n_hrm = n_hrm;
@@ -479,6 +500,7 @@ extern "C" int cosa_proxy_noalloc(const cosa_shape_t* shape, const void* q, cons
   sa.head_dim = shape->head_dim;
   sa.block_size = shape->block_size;
   sa.nqb_total = shape->total_qblocks;
+  sa.nkb_total = total_kblocks(*shape);
   sa.kmax = kmax;
   sa.bp = bp;
   sa.npow2_max = next_pow2(ceil_div(shape->max_seqlen, shape->block_size));

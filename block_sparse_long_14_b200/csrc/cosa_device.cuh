@@ -43,6 +43,29 @@ __device__ __forceinline__ int find_seq(const int32_t* __restrict__ cu, int batc
   return lo;
 }
 
+// Where sequence s sits.  Prefill may follow a cached prefix: the sequence
+// has L keys, its last L - off tokens are the queries (packed in q/out from
+// cu_seqlens[s]), and query rows keep their absolute positions, so position
+// p >= off lives in packed row q_row0 + p.  q-blocks stay on the key-block
+// grid; the first present one is i0 = off / b.  kv_lens == nullptr: every
+// token is a query (off = 0).
+struct SeqSpan {
+  int L, off, i0;
+  long q_row0;
+};
+
+__device__ __forceinline__ SeqSpan seq_span(const int32_t* __restrict__ cu_seqlens,
+                                            const int32_t* __restrict__ kv_lens, int s, int b) {
+  const int q0 = __ldg(cu_seqlens + s);
+  const int lq = __ldg(cu_seqlens + s + 1) - q0;
+  SeqSpan sp;
+  sp.L = kv_lens != nullptr ? __ldg(kv_lens + s) : lq;
+  sp.off = sp.L - lq;
+  sp.i0 = sp.off >= 0 ? sp.off / b : 0;
+  sp.q_row0 = static_cast<long>(q0) - sp.off;
+  return sp;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

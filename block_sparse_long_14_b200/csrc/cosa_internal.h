@@ -17,7 +17,8 @@ struct KPoolArgs {
   const __nv_bfloat16* k_pages;
   const int32_t* page_table;
   const int32_t* cu_seqlens;
-  const int32_t* cu_qblocks;
+  const int32_t* kv_lens;      // nullable: key counts after a cached prefix (else the query counts)
+  const int32_t* cu_kblocks;   // key-block offset of each sequence
   int8_t* kq;     // [Hkv, NKB, d]
   float* ks;      // [Hkv, NKB]
   Status* status;
@@ -27,10 +28,12 @@ struct KPoolArgs {
 
 struct ScoreArgs {
   const __nv_bfloat16* q;
-  const int8_t* kq;
-  const float* ks;
+  const int8_t* kq;    // [Hkv, NKB, d]
+  const float* ks;     // [Hkv, NKB]
   const int32_t* cu_seqlens;
   const int32_t* cu_qblocks;
+  const int32_t* kv_lens;      // nullable, as in KPoolArgs
+  const int32_t* cu_kblocks;
   int32_t* order;
   int32_t* count;
   int32_t* n_hrm;
@@ -38,6 +41,7 @@ struct ScoreArgs {
   Status* status;
   int8_t* qa;          // pooled int8 query vectors [Hq, NQB, R + 1, d] (two-stage path only)
   int batch, num_q_heads, num_kv_heads, head_dim, block_size, nqb_total, kmax, bp, npow2_max;
+  int nkb_total;       // key blocks of the batch (= nqb_total without a cached prefix)
   int scratch_bytes;   // radix-select scratch of the select kernel
 };
 
@@ -47,6 +51,7 @@ struct RemapArgs {
   const int32_t* count;
   const int32_t* cu_seqlens;
   const int32_t* cu_qblocks;
+  const int32_t* kv_lens;      // nullable, as in KPoolArgs
   int32_t* pages;
   Status* status;
   int batch, num_q_heads, block_size, page_size, max_pages_per_seq, num_pages, nqb_total, kmax;
@@ -58,6 +63,7 @@ struct OskArgs {
   const int32_t* count;
   const int32_t* cu_seqlens;
   const int32_t* cu_qblocks;
+  const int32_t* kv_lens;      // nullable, as in KPoolArgs
   const __nv_bfloat16* k_pages;
   const __nv_bfloat16* v_pages;
   __nv_bfloat16* out;
@@ -71,7 +77,7 @@ struct OskArgs {
   int nqb_total, kmax;
   float scale_log2;  // log2(e) / sqrt(d)
   float log2_tau;    // log2(tau), -inf for tau = 0
-  int tau_per_seq;   // 1: tau_s = delta / L_s per sequence, log2(tau_s) = log2_delta - log2(L_s)
+  int tau_per_seq;   // 1: tau_s = delta / L_s per sequence (L_s its key count), log2(tau_s) = log2_delta - log2(L_s)
   float log2_delta;  // log2(delta), -inf when the skip is off
   uint32_t wait_limit;
 };

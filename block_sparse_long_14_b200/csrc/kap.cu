@@ -43,11 +43,15 @@ __global__ void __launch_bounds__(256) kpool_kernel(KPoolArgs a) {
   if (item >= static_cast<long>(a.nkb_total) * a.num_kv_heads) return;
   const int J = static_cast<int>(item / a.num_kv_heads);
   const int g = static_cast<int>(item % a.num_kv_heads);
-  const int s = find_seq(a.cu_qblocks, a.batch, J);
-  const int j = J - __ldg(a.cu_qblocks + s);
-  const int L = __ldg(a.cu_seqlens + s + 1) - __ldg(a.cu_seqlens + s);
+  const int s = find_seq(a.cu_kblocks, a.batch, J);
+  const int j = J - __ldg(a.cu_kblocks + s);
+  const int L = seq_span(a.cu_seqlens, a.kv_lens, s, a.block_size).L;
   const int t0 = j * a.block_size;
   const int ntok = min(a.block_size, L - t0);
+  if (ntok <= 0) {   // cu_kblocks disagrees with the key counts
+    if (lane == 0) report(a.status, kErrBounds, 0x101);
+    return;
+  }
 
   float acc[DPL];
 #pragma unroll
@@ -162,9 +166,18 @@ __device__ void bitonic_sort(uint64_t* base, int nseg, int size, int stride) {
 }
 
 // Tile of the proxy: (q-block I, GT query heads h0.. sharing kv head kv).
+// Its query rows are the tile rows [rlo, rhi) (absolute positions i*b + r);
+// rlo > 0 only in the first q-block after a cached prefix.  Row r of the
+// tile is packed q row q_row0 + i*b + r.  kb0: key block 0 of the sequence
+// in the pooled-key arrays.  bad: the offsets disagree with the lengths.
 struct Tile {
-  int I, h0, kv, s, qb0, i, tok0, L, nrows, n, npow2;
+  int I, h0, kv, s, kb0, i, L, rlo, rhi, n, npow2;
+  long q_row0;
+  bool bad;
 };
+
+// Sub-row v (tile rows 16v .. 16v + 15) holds at least one query row.
+__device__ __forceinline__ bool sub_present(const Tile& t, int v) { return v * 16 < t.rhi && v * 16 + 16 > t.rlo; }
 
 template <int GT>
 __device__ __forceinline__ Tile tile_of(const ScoreArgs& a) {
@@ -174,11 +187,14 @@ __device__ __forceinline__ Tile tile_of(const ScoreArgs& a) {
   t.h0 = (static_cast<int>(blockIdx.x) % ngroups) * GT;
   t.kv = t.h0 / (a.num_q_heads / a.num_kv_heads);
   t.s = find_seq(a.cu_qblocks, a.batch, t.I);
-  t.qb0 = __ldg(a.cu_qblocks + t.s);
-  t.i = t.I - t.qb0;
-  t.tok0 = __ldg(a.cu_seqlens + t.s);
-  t.L = __ldg(a.cu_seqlens + t.s + 1) - t.tok0;
-  t.nrows = min(a.block_size, t.L - t.i * a.block_size);
+  const SeqSpan sp = seq_span(a.cu_seqlens, a.kv_lens, t.s, a.block_size);
+  t.kb0 = __ldg(a.cu_kblocks + t.s);
+  t.i = t.I - __ldg(a.cu_qblocks + t.s) + sp.i0;
+  t.L = sp.L;
+  t.q_row0 = sp.q_row0;
+  t.rlo = max(0, sp.off - t.i * a.block_size);
+  t.rhi = min(a.block_size, t.L - t.i * a.block_size);
+  t.bad = sp.off < 0 || t.rlo >= t.rhi;
   t.n = t.i + 1;
   t.npow2 = 1;
   while (t.npow2 < t.n) t.npow2 <<= 1;
@@ -193,14 +209,14 @@ __device__ void pool_tile(const ScoreArgs& a, const Tile& tl, float* subsum, int
   constexpr int COLS = GT * D;
   constexpr int NCHUNK = COLS / 8;       // 16-byte chunks per token row of the head group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = a.block_size, i = tl.i, tok0 = tl.tok0, h0 = tl.h0, nrows = tl.nrows;
+  const int b = a.block_size, i = tl.i, h0 = tl.h0, rlo = tl.rlo, rhi = tl.rhi;
   // sub-row sums 16-row sub-row sums, token by token, fp32
   for (int item = tid; item < R * NCHUNK; item += 256) {
     const int r = item / NCHUNK, ch = item % NCHUNK;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-    const long row0 = static_cast<long>(tok0) + i * b + r * 16;
+    const long row0 = tl.q_row0 + i * b + r * 16;   // rows outside [rlo, rhi) are never read
     const __nv_bfloat16* src = a.q + (row0 * a.num_q_heads + h0) * D + ch * 8;
     const long stride = static_cast<long>(a.num_q_heads) * D;
 #pragma unroll
@@ -208,11 +224,13 @@ __device__ void pool_tile(const ScoreArgs& a, const Tile& tl, float* subsum, int
       uint4 raw[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        if (r * 16 + t0 + t < nrows) raw[t] = __ldg(reinterpret_cast<const uint4*>(src + (t0 + t) * stride));
+        const int rr = r * 16 + t0 + t;
+        if (rr >= rlo && rr < rhi) raw[t] = __ldg(reinterpret_cast<const uint4*>(src + (t0 + t) * stride));
       }
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        if (r * 16 + t0 + t < nrows) {
+        const int rr = r * 16 + t0 + t;
+        if (rr >= rlo && rr < rhi) {
           const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[t]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -226,7 +244,7 @@ __device__ void pool_tile(const ScoreArgs& a, const Tile& tl, float* subsum, int
     for (int e = 0; e < 8; ++e) subsum[r * COLS + ch * 8 + e] = acc[e];
   }
   for (int x = tid; x < GT * 16 * D / 4; x += 256) reinterpret_cast<uint32_t*>(amat)[x] = 0u;
-  if (tid < R) sub_valid[tid] = (tid * 16 < nrows) ? 1 : 0;
+  if (tid < R) sub_valid[tid] = sub_present(tl, tid) ? 1 : 0;
   __syncthreads();
 
   // block sum (fold of the sub-row sums) and int8 quantisation
@@ -482,7 +500,7 @@ __device__ void select_tile(const ScoreArgs& a, const Tile& tl, const int8_t* am
   constexpr int QR = QB / 4;             // ... as 32-bit registers
   constexpr int KSTEPS = D / 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = tl.n, npow2 = tl.npow2, kv = tl.kv, qb0 = tl.qb0;
+  const int n = tl.n, npow2 = tl.npow2, kv = tl.kv, kb0 = tl.kb0;
   for (int x = tid; x < GT * npow2; x += 256) keys[(x / npow2) * a.npow2_max + (x % npow2)] = ~0ull;
   __syncthreads();
 
@@ -505,8 +523,8 @@ __device__ void select_tile(const ScoreArgs& a, const Tile& tl, const int8_t* am
     best_s[mt][0] = best_s[mt][1] = -FLT_MAX;
     best_j[mt][0] = best_j[mt][1] = 0x7FFFFFFF;
   }
-  const int8_t* kq = a.kq + (static_cast<long>(kv) * a.nqb_total + qb0) * D;
-  const float* ksp = a.ks + static_cast<long>(kv) * a.nqb_total + qb0;
+  const int8_t* kq = a.kq + (static_cast<long>(kv) * a.nkb_total + kb0) * D;
+  const float* ksp = a.ks + static_cast<long>(kv) * a.nkb_total + kb0;
   const int ntiles = (n + 7) >> 3;
   // key fragments and scales of a tile of 8 keys (zeros past n); fetched one tile ahead
   auto load_tile = [&](int tl, uint32_t (&bf)[QR], float& s0, float& s1) {
@@ -675,7 +693,7 @@ __global__ void __launch_bounds__(256, 3) kap_select_tc_kernel(const __grid_cons
   float* sKs = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(bars) + 64);   // [npow2_max] key scales
 
   const Tile tl = tile_of<GT>(a);
-  if (tl.npow2 > a.npow2_max) {
+  if (tl.npow2 > a.npow2_max || tl.bad) {
     if (threadIdx.x == 0) report(a.status, kErrBounds, 0x203);
     return;
   }
@@ -691,7 +709,7 @@ __global__ void __launch_bounds__(256, 3) kap_select_tc_kernel(const __grid_cons
     tmem_relinquish();
   }
   const int ntiles = (n + kTcN - 1) / kTcN;
-  const int row0 = tl.kv * a.nqb_total + tl.qb0;   // Kq row of key block 0 of this sequence
+  const int row0 = tl.kv * a.nkb_total + tl.kb0;   // Kq row of key block 0 of this sequence
   // key tiles cycle through a ring of kTcRing shared-memory slots (b_full[slot]);
   // accumulators alternate between two TMEM buffers (mma_done[t & 1])
   uint64_t* b_full = bars;
@@ -717,7 +735,7 @@ __global__ void __launch_bounds__(256, 3) kap_select_tc_kernel(const __grid_cons
   }
   for (int x = tid; x < GT * npow2; x += 256) keys[(x / npow2) * a.npow2_max + (x % npow2)] = ~0ull;
   {
-    const float* ks_row = a.ks + static_cast<long>(tl.kv) * a.nqb_total + tl.qb0;
+    const float* ks_row = a.ks + static_cast<long>(tl.kv) * a.nkb_total + tl.kb0;
     for (int x = tid; x < n; x += 256) sKs[x] = __ldg(ks_row + x);
   }
   fence_proxy_async();
@@ -799,7 +817,7 @@ __global__ void __launch_bounds__(256, 3) kap_select_tc_kernel(const __grid_cons
     const float s2 = red_s[(GT + mt) * 16 + vv + 1];
     const int j2 = red_j[(GT + mt) * 16 + vv + 1];
     if (better(s2, j2, sv, jv)) { sv = s2; jv = j2; }
-    if (vv * 16 < tl.nrows && jv < n)
+    if (sub_present(tl, vv) && jv < n)
       atomicAnd(reinterpret_cast<unsigned long long*>(&keys[mt * a.npow2_max + jv]), ~(1ull << 63));
   }
   tc_fence_before();
@@ -823,7 +841,7 @@ __global__ void __launch_bounds__(256, 2) kap_score_select_kernel(ScoreArgs a) {
   int* sub_valid = red_j + 8 * GT * 16;                                 // [R]
   uint64_t* keys = reinterpret_cast<uint64_t*>(sub_valid + 16);         // [GT][npow2_max]
   const Tile tl = tile_of<GT>(a);
-  if (tl.npow2 > a.npow2_max) {  // host sizing guarantees this cannot happen
+  if (tl.npow2 > a.npow2_max || tl.bad) {  // host sizing guarantees npow2 fits
     if (threadIdx.x == 0) report(a.status, kErrBounds, 0x200);
     return;
   }
@@ -843,6 +861,10 @@ __global__ void __launch_bounds__(256, 3) qpool_kernel(ScoreArgs a) {
   int8_t* amat = reinterpret_cast<int8_t*>(subsum + R * COLS);          // [GT][16][D]
   int* sub_valid = reinterpret_cast<int*>(amat + GT * 16 * D);          // [R]
   const Tile tl = tile_of<GT>(a);
+  if (tl.bad) {
+    if (threadIdx.x == 0) report(a.status, kErrBounds, 0x204);
+    return;
+  }
   pool_tile<D, GT, R>(a, tl, subsum, amat, sub_valid);
   constexpr int CH = (R + 1) * D / 16;   // 16-byte chunks per head
   for (int x = threadIdx.x; x < GT * CH; x += 256) {
@@ -864,7 +886,7 @@ __global__ void __launch_bounds__(256, 2) kap_select_kernel(ScoreArgs a) {
   uint64_t* keys = reinterpret_cast<uint64_t*>(sub_valid + 16);         // [GT][npow2_max]
   unsigned char* scratch = reinterpret_cast<unsigned char*>(keys + GT * a.npow2_max);
   const Tile tl = tile_of<GT>(a);
-  if (tl.npow2 > a.npow2_max) {
+  if (tl.npow2 > a.npow2_max || tl.bad) {
     if (threadIdx.x == 0) report(a.status, kErrBounds, 0x202);
     return;
   }
@@ -877,7 +899,7 @@ __global__ void __launch_bounds__(256, 2) kap_select_kernel(ScoreArgs a) {
                     a.qa + ((static_cast<long>(tl.h0 + mt) * a.nqb_total + tl.I) * (R + 1) + row) * D) + c);
     reinterpret_cast<uint4*>(amat + (mt * 16 + row) * D)[c] = v;
   }
-  if (threadIdx.x < R) sub_valid[threadIdx.x] = (static_cast<int>(threadIdx.x) * 16 < tl.nrows) ? 1 : 0;
+  if (threadIdx.x < R) sub_valid[threadIdx.x] = sub_present(tl, static_cast<int>(threadIdx.x)) ? 1 : 0;
   __syncthreads();
   select_tile<D, GT, R>(a, tl, amat, sub_valid, red_s, red_j, keys, scratch, a.scratch_bytes);
 }

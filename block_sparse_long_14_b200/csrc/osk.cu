@@ -172,12 +172,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int I = a.nqb_total - 1 - rem / G;
   const int h = g * G + rem % G;
   const int s = find_seq(a.cu_qblocks, a.batch, I);
-  const int i = I - __ldg(a.cu_qblocks + s);
-  const int tok0 = __ldg(a.cu_seqlens + s);
-  const int L = __ldg(a.cu_seqlens + s + 1) - tok0;
   const int b = a.block_size;
-  const int nrows = min(b, L - i * b);
+  // rows of this tile: absolute positions i*b + r, present for r in [rlo, rhi)
+  // (rlo > 0 only in the first q-block after a cached prefix); row r is
+  // packed q/out row q_row0 + i*b + r
+  const SeqSpan sp = seq_span(a.cu_seqlens, a.kv_lens, s, b);
+  const int i = I - __ldg(a.cu_qblocks + s) + sp.i0;
+  const long q_row0 = sp.q_row0;
+  const int L = sp.L;
+  const int rlo = max(0, sp.off - i * b);
+  const int rhi = min(b, L - i * b);
   const int nkb = (L + b - 1) / b;
+  if (sp.off < 0 || rlo >= rhi) {   // offsets disagree with the lengths: nothing is touched
+    if (tid == 0) report(a.status, kErrBounds, 0x302);
+    return;
+  }
   // skip threshold of this sequence: one tau, or tau_s = delta / L_s
   const float log2_tau = a.tau_per_seq ? a.log2_delta - log2f(static_cast<float>(L)) : a.log2_tau;
   const long row_id = static_cast<long>(h) * a.nqb_total + I;
@@ -213,7 +222,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       prefetch_tmap(&vmap);
       mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) tma_load_3d(sQ + c * (kBQ * 128), &qmap, &bars->q_full, c * 64, h, tok0 + i * b);
+      // a negative or past-the-end row coordinate reads zeros; those rows are not present
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sQ + c * (kBQ * 128), &qmap, &bars->q_full, c * 64, h, static_cast<int>(q_row0 + i * b));
     }
   }
   if (warp == kMmaWarp) {
@@ -227,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (n == 0) {
     // nothing listed: zero rows, zero counts
-    if (tid < nrows) {
-      uint4* dst = reinterpret_cast<uint4*>(a.out + ((static_cast<long>(tok0) + i * b + tid) * a.num_q_heads + h) * D);
+    if (tid >= rlo && tid < rhi) {
+      uint4* dst = reinterpret_cast<uint4*>(a.out + ((q_row0 + i * b + tid) * a.num_q_heads + h) * D);
       for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (tid == 0) { a.visited[row_id] = 0; a.skipped[row_id] = 0; }
@@ -383,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;                 // tile row = TMEM lane
     const int col0 = half * C::HALF;                // first key column of this thread
-    const bool row_valid = r < nrows;
+    const bool row_valid = r >= rlo && r < rhi;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float sl2 = a.scale_log2;
     float m = -INFINITY, mref = -INFINITY, l = 0.0f;
@@ -545,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ncomp == 0) {
       // a keep mask that leaves nothing of the row: zero output, like an empty list
       if (row_valid) {
-        uint4* dst = reinterpret_cast<uint4*>(a.out + ((static_cast<long>(tok0) + i * b + r) * a.num_q_heads + h) * D +
+        uint4* dst = reinterpret_cast<uint4*>(a.out + ((q_row0 + i * b + r) * a.num_q_heads + h) * D +
                                               half * (D / 2));
         for (int q4 = 0; q4 < D / 16; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -553,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       const float lrow = half_l[0][r] + half_l[1][r];
       const float inv_l = (row_valid && lrow > 0.0f) ? 1.0f / lrow : 0.0f;
-      __nv_bfloat16* dst = a.out + ((static_cast<long>(tok0) + i * b + r) * a.num_q_heads + h) * D + half * (D / 2);
+      __nv_bfloat16* dst = a.out + ((q_row0 + i * b + r) * a.num_q_heads + h) * D + half * (D / 2);
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         float ov[32];

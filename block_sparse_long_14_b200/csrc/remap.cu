@@ -23,7 +23,7 @@ __global__ void __launch_bounds__(256) remap_kernel(RemapArgs a) {
     int out = -1;
     if (t < __ldg(a.count + row)) {
       const int s = find_seq(a.cu_qblocks, a.batch, I);
-      const int L = __ldg(a.cu_seqlens + s + 1) - __ldg(a.cu_seqlens + s);
+      const int L = seq_span(a.cu_seqlens, a.kv_lens, s, a.block_size).L;   // key count
       const int nkb = (L + a.block_size - 1) / a.block_size;
       const int j = __ldg(a.order + row * a.kmax + t);
       if (j < 0 || j >= nkb) {

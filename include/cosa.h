@@ -58,7 +58,9 @@ typedef enum cosa_status {
 } cosa_status;
 
 /*
- * Shape of one packed prefill batch (query length == key length per sequence).
+ * Shape of one packed prefill batch.  By default every token of a sequence is
+ * a query (query length == key length); with kv_lens set, each sequence's
+ * first tokens are a cached prefix that has keys and values but no queries.
  *
  *   batch              number of sequences B >= 1
  *   num_q_heads        Hq; num_kv_heads Hkv; Hq % Hkv == 0 (GQA group G = Hq/Hkv <= 8).
@@ -78,8 +80,30 @@ typedef enum cosa_status {
  *                      COSA_PAGES_NHD ([P, b_p, Hkv, d]); both read through
  *                      the same page_table
  *
+ * Prefill after a cached prefix (q_len < kv_len; the pages treat full
+ * prefill only, this follows the plainest reading).  kv_lens[s] = L_s is the
+ * key count of sequence s; its queries are its last Lq_s tokens, with
+ * Lq_s = cu_seqlens[s+1] - cu_seqlens[s] and 1 <= Lq_s <= L_s, so query t
+ * sits at position off_s + t, off_s = L_s - Lq_s, and attends to keys
+ * 0 .. off_s + t.  q-blocks stay on the key-block grid: q-block i covers
+ * positions [i*b, (i+1)*b) within [off_s, L_s); the q-blocks wholly inside
+ * the prefix have no list row, and the first present one, floor(off_s / b),
+ * may lack its leading rows (its pooled sums run over its present rows).
+ * With kv_lens set:
+ *   total_tokens   = sum of Lq_s (rows of q and out)
+ *   cu_qblocks     counts the present q-blocks: ceil(L_s/b) - floor(off_s/b)
+ *   total_qblocks  = NQB, their sum (rows of every per-row list)
+ *   cu_kblocks     key-block offsets: ceil(L_s/b) per sequence
+ *   total_kblocks  = NKB, their sum
+ *   max_seqlen     = max L_s (the longest key sequence; sizes kmax)
+ * Every list entry, key block index and page_table row refers to the whole
+ * sequence (prefix included).  kv_lens NULL: L_s = Lq_s and the key blocks
+ * are the q-blocks.
+ *
  * The host fields must agree with the device arrays; the kernels trust them
- * for grid sizes and check every derived index against them.
+ * for grid sizes and check every derived index against them (a tile whose
+ * offsets contradict the lengths is skipped and reported as
+ * COSA_ERR_DEVICE).
  */
 typedef struct cosa_shape {
   int32_t batch;
@@ -96,6 +120,9 @@ typedef struct cosa_shape {
   const int32_t* cu_seqlens;
   const int32_t* cu_qblocks;
   int32_t page_layout;   /* COSA_PAGES_HND or COSA_PAGES_NHD */
+  const int32_t* kv_lens;     /* NULL, or device int32 [B]: keys per sequence (see below) */
+  const int32_t* cu_kblocks;  /* device int32 [B+1] when kv_lens is set, else ignored */
+  int32_t total_kblocks;      /* NKB when kv_lens is set, else ignored */
 } cosa_shape_t;
 
 /* Page pool layouts of k_pages / v_pages. */
@@ -172,7 +199,8 @@ COSA_API int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_
  * key scratch lives instead in one static device array of
  * COSA_NOALLOC_SCRATCH_BYTES bytes that every GPU loading this library holds
  * until the process exits.  Limit: shapes whose pooled keys need more
- * (num_kv_heads * total_qblocks * (head_dim + 4) bytes, plus alignment) are
+ * (num_kv_heads * NKB * (head_dim + 4) bytes, plus alignment; NKB = total_qblocks
+ * without a cached prefix) are
  * rejected with COSA_ERR_WORKSPACE before anything is enqueued.
  *
  * The first call on a device (with that device current) looks up the array's
@@ -211,6 +239,7 @@ COSA_API int cosa_remap(const cosa_shape_t* shape, const int32_t* page_table, co
  *            tau = 0 never skips; the first visited block is never skipped.
  * Outputs (device):
  *   out      bf16 [T, Hq, d] = (sum over kept blocks of exp(s - m) V) / l
+ *            (T = total_tokens: one row per query)
  *   visited  int32 [Hq, NQB]: blocks whose QK^T was computed (= count)
  *   skipped  int32 [Hq, NQB]: visited blocks whose value side was skipped
  *   skipbits uint8 [Hq, NQB, kmax] or NULL: 1 where list entry t was skipped
@@ -225,8 +254,8 @@ COSA_API int cosa_attn(const cosa_shape_t* shape, const void* q, const void* k_p
 /*
  * OSK attention with the pages' length-adaptive threshold (§5.1
  * "Hyperparameters", Appendix D.1 "CoSA settings"): each sequence s of the
- * batch uses tau_s = delta / L_s, L_s its length in tokens, computed on the
- * device from cu_seqlens.  delta = -1 turns the skip off (tau = 0 for every
+ * batch uses tau_s = delta / L_s, L_s its length in tokens (its key count,
+ * the cached prefix included), computed on the device.  delta = -1 turns the skip off (tau = 0 for every
  * sequence); otherwise delta must be > 0.  tau_s >= 1 (a sequence shorter
  * than delta) is applied as written: the skip test compares against
  * ln(tau_s) >= 0.  All other arguments, outputs and errors as cosa_attn.

@@ -21,13 +21,24 @@ MEAN_ABS = 2e-3
 DELTA_WINDOW = 1e-3
 
 
-def upload(w, device="cuda"):
+def prefix_q(w, q_lens):
+    """Packed Q of prefill after a cached prefix: each sequence's last q_len rows."""
+    parts, tok0 = [], 0
+    for L, Lq in zip(w.seqlens, q_lens):
+        parts.append(w.q[tok0 + L - Lq:tok0 + L])
+        tok0 += L
+    return np.ascontiguousarray(np.concatenate(parts, axis=0))
+
+
+def upload(w, device="cuda", q_lens=None):
+    """Device copies of a workload; with q_lens, only the query rows of Q."""
     def bf16(x):
         return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(device)
 
     batch = cosa.Batch(w.seqlens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.page_size,
-                       w.num_pages, w.max_pages_per_seq, device=device)
-    return dict(batch=batch, q=bf16(w.q), k_pages=bf16(w.k_pages), v_pages=bf16(w.v_pages),
+                       w.num_pages, w.max_pages_per_seq, device=device, q_lens=q_lens)
+    q = w.q if q_lens is None else prefix_q(w, q_lens)
+    return dict(batch=batch, q=bf16(q), k_pages=bf16(w.k_pages), v_pages=bf16(w.v_pages),
                 page_table=torch.from_numpy(np.ascontiguousarray(w.page_table)).to(device))
 
 
@@ -58,9 +69,11 @@ def assert_proxy_equal(got, ref, rows=None):
                                  f"gpu {g[tuple(bad[0])]} vs oracle {r[tuple(bad[0])]}")
 
 
-def compare_attn(res, ref, w, tau, units):
+def compare_attn(res, ref, w, tau, units, q_lens=None):
     """Compare GPU OSK results with the oracle on the given (h, I) units.
 
+    q_lens: per-sequence query counts of prefill after a cached prefix (rows
+    and list rows then cover only the queries).
     Returns a dict of statistics; raises AssertionError on a violation.
     """
     out = res["out"].float().cpu().numpy()
@@ -69,16 +82,19 @@ def compare_attn(res, ref, w, tau, units):
     skipbits = res["skipbits"].cpu().numpy().astype(bool)
     b = w.block_size
     log_tau = math.log(tau) if tau > 0 else -math.inf
-    seq_of, tok0 = [], [0]
-    for s, L in enumerate(w.seqlens):
-        seq_of += [s] * ((L + b - 1) // b)
-        tok0.append(tok0[-1] + L)
-    blk0 = np.concatenate([[0], np.cumsum([(L + b - 1) // b for L in w.seqlens])])
+    q_lens = list(w.seqlens) if q_lens is None else list(q_lens)
+    seq_of, tok0, nq = [], [0], []
+    for s, (L, Lq) in enumerate(zip(w.seqlens, q_lens)):
+        nq.append((L + b - 1) // b - (L - Lq) // b)           # q-blocks holding a query row
+        seq_of += [s] * nq[-1]
+        tok0.append(tok0[-1] + Lq)
+    blk0 = np.concatenate([[0], np.cumsum(nq)])
     errs, n_el, max_err, exempt_units, n_skip = 0.0, 0, 0.0, 0, 0
     for h, I in units:
         s = seq_of[I]
-        i = I - blk0[s]
         L = w.seqlens[s]
+        off = L - q_lens[s]
+        i = I - blk0[s] + off // b
         k = int(ref["visited"][h, I])
         assert visited[h, I] == k, f"visited[{h},{I}] {visited[h, I]} != {k}"
         gs, rs = skipbits[h, I, :k], ref["skip"][h, I, :k]
@@ -93,7 +109,7 @@ def compare_attn(res, ref, w, tau, units):
             continue
         assert skipped[h, I] == int(gs.sum())
         n_skip += int(gs.sum())
-        rows = slice(tok0[s] + i * b, tok0[s] + min(L, (i + 1) * b))
+        rows = slice(tok0[s] + max(off, i * b) - off, tok0[s] + min(L, (i + 1) * b) - off)
         e = np.abs(out[rows, h].astype(np.float64) - ref["out"][rows, h])
         assert np.isfinite(out[rows, h]).all()
         max_err = max(max_err, float(e.max()))

@@ -136,3 +136,41 @@ def test_page_layouts(lib):
     assert _ws(_shape(page_layout=1), 0.1)[0] > 0
     assert _ws(_shape(page_layout=2), 0.1)[0] == 0
     assert lib.cosa_version() >= 101
+
+
+def test_cached_prefix_shape_checks(lib):
+    """kv_lens set: the key blocks are counted apart from the q-blocks, the
+    workspace's pooled keys follow NKB, and inconsistent counts are refused."""
+    # 128K keys, the last 8K tokens are queries: 64 present q-blocks of 1024 key blocks
+    ok = dict(total_tokens=8192, total_qblocks=64, max_seqlen=131072, kv_lens=48, cu_kblocks=64,
+              total_kblocks=1024)
+    n_prefix, kmax = _ws(_shape(**ok), 0.05)
+    assert kmax == kap.kmax_for(1024, 0.05)          # lists sized by the longest key sequence
+    n_full, _ = _ws(_shape(), 0.05)
+    # pooled keys and scales sized by NKB (same as full prefill); query vectors by NQB only
+    qa_full = 32 * 1024 * 9 * 128
+    qa_prefix = 32 * 64 * 9 * 128
+    assert n_full - n_prefix == qa_full - qa_prefix
+    for bad in (dict(cu_kblocks=0), dict(total_kblocks=0), dict(total_kblocks=1023), dict(total_kblocks=63,
+                max_seqlen=8000)):
+        assert _ws(_shape(**{**ok, **bad}), 0.05)[0] == 0, bad
+    # without kv_lens the old rule holds: every token a query, max_seqlen <= total_tokens
+    assert _ws(_shape(total_tokens=8192, total_qblocks=64, max_seqlen=131072), 0.05)[0] == 0
+    assert lib.cosa_version() >= 102
+
+
+def test_batch_prefix_offsets_on_the_host():
+    """Batch's offset arrays for a cached prefix, checked on the CPU."""
+    b = cosa.Batch([300, 128, 133], 4, 2, 64, 64, 16, 64, 8, device="cpu", q_lens=[100, 128, 1])
+    assert b.cu_seqlens.tolist() == [0, 100, 228, 229]
+    # q-blocks holding a query row: 5 - 200//64, 2 - 0, 3 - 132//64
+    assert b.cu_qblocks.tolist() == [0, 2, 4, 5]
+    assert b.cu_kblocks.tolist() == [0, 5, 7, 10]
+    assert b.kv_lens.tolist() == [300, 128, 133]
+    assert (b.total_tokens, b.total_qblocks, b.total_kblocks) == (229, 5, 10)
+    assert b.c.total_kblocks == 10 and b.c.max_seqlen == 300
+    full = cosa.Batch([300, 128], 4, 2, 64, 64, 16, 64, 8, device="cpu")
+    assert full.kv_lens is None and full.c.kv_lens is None and full.c.total_kblocks == 0
+    for bad in ([0, 128, 1], [301, 128, 1], [1, 1]):
+        with pytest.raises(ValueError):
+            cosa.Batch([300, 128, 133], 4, 2, 64, 64, 16, 64, 8, device="cpu", q_lens=bad)

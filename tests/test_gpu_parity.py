@@ -235,3 +235,53 @@ def test_repeated_calls_are_deterministic():
         outs.append((sel["order"].clone(), r["out"].clone(), r["skipped"].clone()))
     for o in outs[1:]:
         assert torch.equal(o[0], outs[0][0]) and torch.equal(o[1], outs[0][1]) and torch.equal(o[2], outs[0][2])
+
+
+# Prefill after a cached prefix: queries are each sequence's last q_len tokens.
+# Prefixes on and off the block grid, two whole sub-rows absent, single-query
+# sequences, and the d = 64 proxy path.
+PREFIX_CASES = {
+    "ragged_b128_p64": [1000 - 384, 300, 2100 - 1000, 1],
+    "b64_g8": [900 - 100, 200 - 163],
+    "short_seqs": [50, 1, 1, 64],
+    "d64_b128_p32": [1200 - 256, 513 - 200],
+}
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_prefix(name, budget):
+    w, q_lens = workload(name), PREFIX_CASES[name]
+    return kap.kap_proxy(gu.prefix_q(w, q_lens), w.k_pages, w.page_table, w.seqlens, w.num_kv_heads,
+                         w.block_size, budget, q_lens=q_lens)
+
+
+@pytest.mark.parametrize("budget,tau", [(0.25, 1e-3), (1.0, 0.0)])
+@pytest.mark.parametrize("name", list(PREFIX_CASES))
+def test_prefix_prefill_matches_oracle(name, budget, tau):
+    """Proxy lists (workspace and allocation-free paths) and remap bit-exact,
+    attention within tolerance, for prefill after a cached prefix."""
+    w, q_lens = workload(name), PREFIX_CASES[name]
+    d = gu.upload(w, q_lens=q_lens)
+    got, kmax, ws = gu.run_proxy(d, budget)
+    ref = oracle_prefix(name, budget)
+    assert kmax == ref["kmax"]
+    gu.assert_proxy_equal(got, ref)
+    na = cosa.proxy_noalloc(d["batch"], d["q"], d["k_pages"], d["page_table"], budget, kmax)
+    torch.cuda.synchronize()
+    gu.assert_proxy_equal({k: v.cpu().numpy() for k, v in na.items()}, ref)
+    sel = {k: torch.from_numpy(v).cuda() for k, v in got.items()}
+    pages = cosa.remap(d["batch"], d["page_table"], sel["order"], sel["count"], kmax)
+    expect = kap.remap(ref["order"], ref["count"], w.page_table, w.seqlens, w.block_size, w.page_size,
+                       q_lens=q_lens)
+    assert np.array_equal(pages.cpu().numpy(), expect)
+    res = gu.run_attn(d, sel, kmax, tau, ws)
+    qp = gu.prefix_q(w, q_lens)
+    o = osk.osk(qp, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, ref["order"],
+                ref["count"], tau, q_lens=q_lens)
+    units = [(h, I) for h in range(w.num_q_heads) for I in range(ref["count"].shape[1])]
+    stats = gu.compare_attn(res, o, w, tau, units, q_lens=q_lens)
+    if budget == 1.0 and tau == 0.0:
+        dn = dense.dense_causal(qp, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, q_lens=q_lens)
+        err = np.abs(res["out"].float().cpu().numpy() - dn)
+        assert err.max() <= gu.MAX_ABS and err.mean() <= gu.MEAN_ABS
+    print(name, budget, tau, stats)
