@@ -20,7 +20,7 @@ import os
 import torch
 
 __all__ = [
-    "Batch", "CosaError", "PAGES_HND", "PAGES_NHD", "alloc_workspace", "attn", "attn_delta", "attn_masked", "check", "lib", "proxy", "remap",
+    "Batch", "CosaError", "PAGES_HND", "PAGES_NHD", "alloc_workspace", "attn", "attn_delta", "attn_masked", "check", "lib", "proxy", "proxy_top_p", "remap",
     "set_wait_limit", "tau_from_delta", "workspace_size", "LIB_PATH",
 ]
 
@@ -61,6 +61,8 @@ _SIGS = {
                                   _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "cosa_proxy_noalloc": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, ctypes.c_float, ctypes.c_int32,
                                           _P, _P, _P, _P, _P]),
+    "cosa_proxy_top_p": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, ctypes.c_float, ctypes.c_int32,
+                                        _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "cosa_remap": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, ctypes.c_int32, _P, _P]),
     "cosa_attn": (ctypes.c_int, [ctypes.POINTER(_Shape), _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_float,
                                  _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -189,6 +191,26 @@ def proxy(batch: Batch, q, k_pages, page_table, budget: float, kmax: int, worksp
                            _ptr(out["n_hrm"], torch.int32, "n_hrm"), _ptr(out["hrm"], torch.uint8, "hrm"),
                            _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream())
     _check(rc, "cosa_proxy")
+    return out
+
+
+def proxy_top_p(batch: Batch, q, k_pages, page_table, p: float, kmax: int, workspace, out=None):
+    """KAP with the Top-p stage-1 cut (cosa_proxy_top_p).  kmax must cover
+    every candidate: alloc_workspace(batch, 1.0) returns it."""
+    H, N = batch.num_q_heads, batch.total_qblocks
+    dev = q.device
+    if out is None:
+        out = dict(order=torch.empty((H, N, kmax), dtype=torch.int32, device=dev),
+                   count=torch.empty((H, N), dtype=torch.int32, device=dev),
+                   n_hrm=torch.empty((H, N), dtype=torch.int32, device=dev),
+                   hrm=torch.empty((H, N, kmax), dtype=torch.uint8, device=dev))
+    rc = _lib().cosa_proxy_top_p(ctypes.byref(batch.c), _ptr(q, torch.bfloat16, "q"),
+                                 _ptr(k_pages, torch.bfloat16, "k_pages"), _ptr(page_table, torch.int32, "page_table"),
+                                 ctypes.c_float(p), int(kmax), _ptr(out["order"], torch.int32, "order"),
+                                 _ptr(out["count"], torch.int32, "count"), _ptr(out["n_hrm"], torch.int32, "n_hrm"),
+                                 _ptr(out["hrm"], torch.uint8, "hrm"), _ptr(workspace, torch.uint8, "workspace"),
+                                 workspace.numel(), _stream())
+    _check(rc, "cosa_proxy_top_p")
     return out
 
 

@@ -77,9 +77,10 @@ int total_kblocks(const cosa_shape_t& s) { return s.kv_lens != nullptr ? s.total
 const int32_t* cu_kblocks(const cosa_shape_t& s) { return s.kv_lens != nullptr ? s.cu_kblocks : s.cu_qblocks; }
 
 // Workspace: status block, pooled int8 keys [Hkv, NKB, d], key scales
-// [Hkv, NKB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d].
+// [Hkv, NKB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d], and the
+// q-block vectors' max-abs [Hq, NQB] (the Top-p cut's logit scale).
 struct WsLayout {
-  size_t kq_off, ks_off, qa_off, total;
+  size_t kq_off, ks_off, qa_off, qm_off, total;
 };
 
 WsLayout ws_layout(const cosa_shape_t& s) {
@@ -90,7 +91,8 @@ WsLayout ws_layout(const cosa_shape_t& s) {
   w.qa_off = align_up(w.ks_off + static_cast<size_t>(s.num_kv_heads) * total_kblocks(s) * 4, 256);
   const size_t qa_bytes =
       static_cast<size_t>(s.num_q_heads) * s.total_qblocks * (s.block_size / 16 + 1) * s.head_dim;
-  w.total = align_up(w.qa_off + qa_bytes, 256);
+  w.qm_off = align_up(w.qa_off + qa_bytes, 256);
+  w.total = align_up(w.qm_off + static_cast<size_t>(s.num_q_heads) * s.total_qblocks * 4, 256);
   return w;
 }
 
@@ -178,17 +180,21 @@ int cosa_workspace_init(void* workspace, size_t ws_bytes, cosa_stream_t stream) 
              : COSA_ERR_CUDA;
 }
 
-int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, const int32_t* page_table, float budget,
-               int32_t kmax, int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags, void* workspace,
-               size_t ws_bytes, cosa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The shared body of cosa_proxy (top_p = 0: the budget cut bp) and
+// cosa_proxy_top_p (bp = 10^4, the Top-p cut at top_p).
+int proxy_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, const int32_t* page_table, int bp,
+               float top_p, int32_t kmax, int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags,
+               void* workspace, size_t ws_bytes, cosa_stream_t stream) {
   int rc = check_shape(shape);
   if (rc != COSA_OK) return rc;
   if (q == nullptr || k_pages == nullptr || page_table == nullptr || order == nullptr || count == nullptr ||
       n_hrm == nullptr || hrm_flags == nullptr || workspace == nullptr)
     return COSA_ERR_INVALID_ARG;
-  if (!(budget > 0.0f && budget <= 1.0f)) return COSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return COSA_ERR_INVALID_ARG;
-  const int bp = budget_bp(budget);
   if (kmax < keep_count(ceil_div(shape->max_seqlen, shape->block_size), bp)) return COSA_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(*shape);
   if (ws_bytes < w.total) return COSA_ERR_WORKSPACE;
@@ -240,6 +246,8 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   sa.bp = bp;
   sa.npow2_max = next_pow2(ceil_div(shape->max_seqlen, shape->block_size));
   sa.qa = reinterpret_cast<int8_t*>(ws + w.qa_off);
+  sa.qm = reinterpret_cast<float*>(ws + w.qm_off);
+  sa.top_p = top_p;
   const int GT = proxy_group(*shape);
   sa.scratch_bytes = select_scratch_bytes(*shape, kmax, GT, sa.npow2_max);
   if (launch_qpool(sa, GT, st) != cudaSuccess) return COSA_ERR_CUDA;
@@ -255,6 +263,26 @@ int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, co
     if (launch_select(sa, GT, st) != cudaSuccess) return COSA_ERR_CUDA;
   }
   return COSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages, const int32_t* page_table, float budget,
+               int32_t kmax, int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags, void* workspace,
+               size_t ws_bytes, cosa_stream_t stream) {
+  if (!(budget > 0.0f && budget <= 1.0f)) return COSA_ERR_INVALID_ARG;
+  return proxy_impl(shape, q, k_pages, page_table, budget_bp(budget), 0.0f, kmax, order, count, n_hrm, hrm_flags,
+                    workspace, ws_bytes, stream);
+}
+
+int cosa_proxy_top_p(const cosa_shape_t* shape, const void* q, const void* k_pages, const int32_t* page_table,
+                     float p, int32_t kmax, int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags,
+                     void* workspace, size_t ws_bytes, cosa_stream_t stream) {
+  if (!(p > 0.0f && p <= 1.0f)) return COSA_ERR_INVALID_ARG;
+  return proxy_impl(shape, q, k_pages, page_table, 10000, p, kmax, order, count, n_hrm, hrm_flags, workspace,
+                    ws_bytes, stream);
 }
 
 int cosa_remap(const cosa_shape_t* shape, const int32_t* page_table, const int32_t* order, const int32_t* count,

@@ -43,6 +43,8 @@ struct ScoreArgs {
   int batch, num_q_heads, num_kv_heads, head_dim, block_size, nqb_total, kmax, bp, npow2_max;
   int nkb_total;       // key blocks of the batch (= nqb_total without a cached prefix)
   int scratch_bytes;   // radix-select scratch of the select kernel
+  float* qm;           // [Hq, NQB] max-abs of each q-block sum vector (written by qpool; nullable)
+  float top_p;         // 0: budget cut k_i from bp; in (0, 1]: Top-p cut (reads qm)
 };
 
 struct RemapArgs {

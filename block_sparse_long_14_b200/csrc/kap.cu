@@ -24,6 +24,9 @@
 //                    workspace holds the pooled queries (the allocation-free
 //                    entry point).
 // Scores are exact integers, so the ordering is reproducible bit for bit.
+// The stage-1 cut is the budget fraction k_i, or the pages' Top-p rule
+// (top_p_emit), which keeps the shortest prefix of the full order holding
+// a fraction p of the row's estimated attention mass.
 #include <cfloat>
 #include <cstdint>
 
@@ -137,6 +140,13 @@ __device__ __forceinline__ uint64_t make_key(float sc, int j) {
   return (1ull << 63) | (static_cast<uint64_t>(~asc) << 31) | static_cast<uint32_t>(j);
 }
 
+// The score a sort key was made from (make_key is a bijection on non-zero
+// floats and maps both zeros to +0).
+__device__ __forceinline__ float score_of_key(uint64_t key) {
+  const uint32_t asc = ~static_cast<uint32_t>(key >> 31);
+  return __uint_as_float((asc & 0x80000000u) ? (asc & 0x7FFFFFFFu) : ~asc);
+}
+
 __device__ __forceinline__ bool better(float s2, int j2, float s1, int j1) {
   return s2 > s1 || (s2 == s1 && j2 < j1);
 }
@@ -205,7 +215,8 @@ __device__ __forceinline__ Tile tile_of(const ScoreArgs& a) {
 // fp32), the q-block sum (their fold), and the int8 quantisation of the
 // (R + 1) vectors of each head into amat [GT][16][D] (rows 0..R; the rest 0).
 template <int D, int GT, int R>
-__device__ void pool_tile(const ScoreArgs& a, const Tile& tl, float* subsum, int8_t* amat, int* sub_valid) {
+__device__ void pool_tile(const ScoreArgs& a, const Tile& tl, float* subsum, int8_t* amat, int* sub_valid,
+                          float* qm_s) {
   constexpr int COLS = GT * D;
   constexpr int NCHUNK = COLS / 8;       // 16-byte chunks per token row of the head group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -272,18 +283,99 @@ __device__ void pool_tile(const ScoreArgs& a, const Tile& tl, float* subsum, int
 #pragma unroll
     for (int e = 0; e < DPL; ++e)
       amat[(hh * 16 + v) * D + lane * DPL + e] = static_cast<int8_t>(rintf(__fmul_rn(x[e], inv)));
+    if (qm_s != nullptr && v == 0 && lane == 0) qm_s[hh] = M;   // the q-block vector's scale
   }
   __syncthreads();
 
+}
+
+// Top-p stage-1 cut of one tile (256 threads; §5.1 "Hyperparameters" and
+// Appendix D.1 give only p, so the mass is this library's reading).  Block
+// j's share of the row's attention is estimated as
+//   w_j = n_tok(j) exp((s_j - s_max) zscale),  zscale = (M_q / 127) / (n_rows sqrt(d)),
+// zscale turning the pooled score s_j back into the mean logit between the
+// q-block's rows and block j's keys (M_q: the q-block sum's max-abs, dropped
+// from the ranking score).  Each head keeps the shortest prefix of its full
+// flag-grouped order whose mass reaches p of the row's total (p = 1: all).
+// One warp per head; fp32 masses summed in one fixed order (a contiguous
+// chunk per lane, then the lanes in order), so the cut is deterministic.
+template <int GT>
+__device__ void top_p_emit(const ScoreArgs& a, const Tile& tl, uint64_t* keys) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = tl.n, b = a.block_size;
+  bitonic_sort(keys, GT, tl.npow2, a.npow2_max);   // ascending keys = visit order; ends with a barrier
+  if (warp >= GT) return;
+  const int mt = warp;
+  const uint64_t* kr = keys + mt * a.npow2_max;
+  int nh = 0;   // HRM keys (bit 63 clear) form the prefix; every lane takes every ballot
+  for (int base = 0; base < n; base += 32) {
+    const int x = base + lane;
+    nh += __popc(__ballot_sync(0xffffffffu, x < n && !(kr[x] >> 63)));
+  }
+  const float s_max = fmaxf(score_of_key(kr[0]), nh < n ? score_of_key(kr[nh]) : -FLT_MAX);
+  const long row = static_cast<long>(tl.h0 + mt) * a.nqb_total + tl.I;
+  const float qm = a.qm[row];
+  const float zscale =
+      __fdiv_rn(__fdiv_rn(qm, 127.0f), __fmul_rn(static_cast<float>(tl.rhi - tl.rlo), sqrtf(static_cast<float>(a.head_dim))));
+  auto mass = [&](uint64_t key) {
+    const int j = static_cast<int>(key & 0x7FFFFFFFu);
+    const float ntok = static_cast<float>(min(b, tl.L - j * b));
+    return __fmul_rn(ntok, expf(__fmul_rn(__fsub_rn(score_of_key(key), s_max), zscale)));
+  };
+  const int c = (n + 31) >> 5;
+  const int lo = min(n, lane * c), hi = min(n, lo + c);
+  float part = 0.0f;
+  for (int x = lo; x < hi; ++x) part = __fadd_rn(part, mass(kr[x]));
+  float inc = part;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc = __fadd_rn(inc, y);
+  }
+  const float total = __shfl_sync(0xffffffffu, inc, 31);
+  float cum = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) cum = 0.0f;
+  int first = n;   // entries kept: the first prefix whose mass reaches p * total (else all)
+  if (a.top_p < 1.0f) {
+    const float target = __fmul_rn(a.top_p, total);
+    for (int x = lo; x < hi; ++x) {
+      cum = __fadd_rn(cum, mass(kr[x]));
+      if (cum >= target) { first = x + 1; break; }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, off));
+  int k = max(1, first);
+  if (k > a.kmax) {   // the host sizes kmax for every candidate; never taken
+    if (lane == 0) report(a.status, kErrBounds, 0x205);
+    k = a.kmax;
+  }
+  const long o = row * a.kmax;
+  for (int t = lane; t < a.kmax; t += 32) {
+    const uint64_t key = t < k ? kr[t] : 0ull;
+    a.order[o + t] = t < k ? static_cast<int32_t>(key & 0x7FFFFFFFu) : -1;
+    a.hrm[o + t] = (t < k && !(key >> 63)) ? 1 : 0;
+  }
+  if (lane == 0) {
+    a.count[row] = k;
+    a.n_hrm[row] = min(nh, k);
+  }
 }
 
 // Selection and output of one tile (256 threads): each head's k_i smallest
 // sort keys of keys [GT][npow2_max] (HRM flags already folded in), in
 // ascending order, written as the visit lists.  `state` holds a few words
 // of per-head radix-select state; `scratch` the histograms and buffers.
-template <int GT, int R>
+// kTopP = false compiles the Top-p cut out (kernels of entry points without it).
+template <int GT, int R, bool kTopP = true>
 __device__ void select_emit(const ScoreArgs& a, const Tile& tl, uint64_t* keys, float* state, unsigned char* scratch,
                             int scratch_bytes) {
+  if constexpr (kTopP) {
+    if (a.top_p > 0.0f) {
+      top_p_emit<GT>(a, tl, keys);
+      return;
+    }
+  }
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = tl.n, npow2 = tl.npow2, h0 = tl.h0, I = tl.I;
   float* red_s = state;
@@ -493,7 +585,7 @@ __device__ void select_emit(const ScoreArgs& a, const Tile& tl, uint64_t* keys, 
 // amat [GT][16][D]: exact integer scores on int8 tensor cores, each sub-row's
 // argmax (the HRM flags), the k_i smallest sort keys, the output lists.
 // `scratch` (scratch_bytes) holds the radix-select histograms and buffers.
-template <int D, int GT, int R>
+template <int D, int GT, int R, bool kTopP = true>
 __device__ void select_tile(const ScoreArgs& a, const Tile& tl, const int8_t* amat, const int* sub_valid,
                             float* red_s, int* red_j, uint64_t* keys, unsigned char* scratch, int scratch_bytes) {
   constexpr int QB = D / 4;              // bytes of a row each MMA quad-lane owns
@@ -613,7 +705,7 @@ __device__ void select_tile(const ScoreArgs& a, const Tile& tl, const int8_t* am
   }
   __syncthreads();
 
-  select_emit<GT, R>(a, tl, keys, red_s, scratch, scratch_bytes);
+  select_emit<GT, R, kTopP>(a, tl, keys, red_s, scratch, scratch_bytes);
 }
 
 // ============================================================ tcgen05 scoring
@@ -845,8 +937,8 @@ __global__ void __launch_bounds__(256, 2) kap_score_select_kernel(ScoreArgs a) {
     if (threadIdx.x == 0) report(a.status, kErrBounds, 0x200);
     return;
   }
-  pool_tile<D, GT, R>(a, tl, subsum, amat, sub_valid);
-  select_tile<D, GT, R>(a, tl, amat, sub_valid, red_s, red_j, keys, reinterpret_cast<unsigned char*>(subsum),
+  pool_tile<D, GT, R>(a, tl, subsum, amat, sub_valid, nullptr);
+  select_tile<D, GT, R, false>(a, tl, amat, sub_valid, red_s, red_j, keys, reinterpret_cast<unsigned char*>(subsum),
                         R * COLS * 4);
 }
 
@@ -860,12 +952,14 @@ __global__ void __launch_bounds__(256, 3) qpool_kernel(ScoreArgs a) {
   float* subsum = reinterpret_cast<float*>(smem);                       // [R][COLS]
   int8_t* amat = reinterpret_cast<int8_t*>(subsum + R * COLS);          // [GT][16][D]
   int* sub_valid = reinterpret_cast<int*>(amat + GT * 16 * D);          // [R]
+  float* qm_s = reinterpret_cast<float*>(sub_valid + 16);               // [GT]
   const Tile tl = tile_of<GT>(a);
   if (tl.bad) {
     if (threadIdx.x == 0) report(a.status, kErrBounds, 0x204);
     return;
   }
-  pool_tile<D, GT, R>(a, tl, subsum, amat, sub_valid);
+  pool_tile<D, GT, R>(a, tl, subsum, amat, sub_valid, qm_s);
+  if (a.qm != nullptr && threadIdx.x < GT) a.qm[static_cast<long>(tl.h0 + threadIdx.x) * a.nqb_total + tl.I] = qm_s[threadIdx.x];
   constexpr int CH = (R + 1) * D / 16;   // 16-byte chunks per head
   for (int x = threadIdx.x; x < GT * CH; x += 256) {
     const int mt = x / CH, c = x % CH;
@@ -911,7 +1005,7 @@ size_t score_smem_bytes(int D, int GT, int R, int npow2_max) {
 }
 
 size_t qpool_smem_bytes(int D, int GT, int R) {
-  return static_cast<size_t>(R) * GT * D * 4 + static_cast<size_t>(GT) * 16 * D + 16 * 4;
+  return static_cast<size_t>(R) * GT * D * 4 + static_cast<size_t>(GT) * 16 * D + 16 * 4 + 4 * 4;
 }
 
 size_t select_smem_bytes(int D, int GT, int npow2_max, int scratch_bytes) {

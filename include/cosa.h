@@ -182,6 +182,31 @@ COSA_API int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_
                int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags,
                void* workspace, size_t ws_bytes, cosa_stream_t stream);
 
+/*
+ * KAP proxy with the pages' Top-p stage-1 rule (§5.1 "Hyperparameters",
+ * Appendix D.1: p = 0.95 for Qwen3-8B, calibrated per context length for
+ * Llama-3.1-8B) instead of a budget fraction.  Scores, HRM flags and the
+ * visit order are those of cosa_proxy; each row keeps the shortest prefix
+ * of its full order (all n_i = i + 1 causal candidates) whose estimated
+ * attention mass reaches p of the row's total.  The pages give p but not the
+ * mass; this library's reading:
+ *   w_j = n_tok(j) * exp((s_j - s_max) * zscale),
+ *   zscale = (M_q / 127) / (n_rows * sqrt(d)),
+ * s_j the block score, M_q the max-abs of the q-block's pooled query sum
+ * (the scale the ranking score drops), n_rows the q-block's query rows, so
+ * s_j * zscale estimates the mean logit between the q-block and block j.
+ * Masses are fp32, summed in one fixed order (deterministic run to run); a
+ * prefix whose share lies within about 1e-5 of p may be cut either way.
+ *   p      in (0, 1]; p = 1 keeps every candidate
+ *   kmax   at least ceil(max_seqlen / b) (cosa_workspace_size with budget
+ *          1.0 returns it): a row may keep every candidate
+ * Outputs, workspace and errors as cosa_proxy; count[h, I] is the row's cut.
+ */
+COSA_API int cosa_proxy_top_p(const cosa_shape_t* shape, const void* q, const void* k_pages,
+                              const int32_t* page_table, float p, int32_t kmax,
+                              int32_t* order, int32_t* count, int32_t* n_hrm, uint8_t* hrm_flags,
+                              void* workspace, size_t ws_bytes, cosa_stream_t stream);
+
 /* Capacity of the static device scratch array behind cosa_proxy_noalloc. */
 #define COSA_NOALLOC_SCRATCH_BYTES (4u << 20)
 

@@ -147,10 +147,10 @@ def test_cached_prefix_shape_checks(lib):
     n_prefix, kmax = _ws(_shape(**ok), 0.05)
     assert kmax == kap.kmax_for(1024, 0.05)          # lists sized by the longest key sequence
     n_full, _ = _ws(_shape(), 0.05)
-    # pooled keys and scales sized by NKB (same as full prefill); query vectors by NQB only
-    qa_full = 32 * 1024 * 9 * 128
-    qa_prefix = 32 * 64 * 9 * 128
-    assert n_full - n_prefix == qa_full - qa_prefix
+    # pooled keys and scales sized by NKB (same as full prefill); query vectors and their
+    # scales by NQB only
+    per_qblock = 32 * 9 * 128 + 32 * 4
+    assert n_full - n_prefix == (1024 - 64) * per_qblock
     for bad in (dict(cu_kblocks=0), dict(total_kblocks=0), dict(total_kblocks=1023), dict(total_kblocks=63,
                 max_seqlen=8000)):
         assert _ws(_shape(**{**ok, **bad}), 0.05)[0] == 0, bad
@@ -174,3 +174,20 @@ def test_batch_prefix_offsets_on_the_host():
     for bad in ([0, 128, 1], [301, 128, 1], [1, 1]):
         with pytest.raises(ValueError):
             cosa.Batch([300, 128, 133], 4, 2, 64, 64, 16, 64, 8, device="cpu", q_lens=bad)
+
+
+def test_proxy_top_p_arguments(lib):
+    """cosa_proxy_top_p: p in (0, 1]; kmax must cover every candidate."""
+    sh = _shape()
+    n_all = 1024
+
+    def call(p, kmax):
+        return lib.cosa_proxy_top_p(ctypes.byref(sh), 16, 16, 16, ctypes.c_float(p), kmax, 16, 16, 16, 16, 256,
+                                    1 << 40, None)
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        assert call(p, n_all) == 1
+    assert call(0.95, n_all - 1) == 1        # a row may keep all of its candidates
+    rc = lib.cosa_proxy_top_p(ctypes.byref(sh), None, None, None, ctypes.c_float(0.95), n_all, None, None, None,
+                              None, None, 0, None)
+    assert rc == 1
+    assert _ws(sh, 1.0)[1] == n_all         # budget 1.0 reports the kmax Top-p needs

@@ -285,3 +285,50 @@ def test_prefix_prefill_matches_oracle(name, budget, tau):
         err = np.abs(res["out"].float().cpu().numpy() - dn)
         assert err.max() <= gu.MAX_ABS and err.mean() <= gu.MEAN_ABS
     print(name, budget, tau, stats)
+
+
+TOP_P_EPS = 1e-5   # a cut whose oracle share lies within this of p may fall on either side
+
+
+@pytest.mark.parametrize("p", [0.5, 0.9, 0.95, 1.0])
+@pytest.mark.parametrize("name", ["tiny", "ragged_b128_p64", "qwen_mix", "d64_b128_p32", "b64_g8"])
+def test_proxy_top_p_matches_oracle(name, p):
+    """The Top-p cut: each row's count within the oracle's window around p,
+    and its entries the leading entries of the full flag-grouped order."""
+    w, d = workload(name), device(name)
+    ws, kmax = cosa.alloc_workspace(d["batch"], 1.0)
+    sel = cosa.proxy_top_p(d["batch"], d["q"], d["k_pages"], d["page_table"], p, kmax, ws)
+    cosa.check(ws)
+    got = {k: v.cpu().numpy() for k, v in sel.items()}
+    ref = kap.kap_proxy_top_p(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, p,
+                              eps=TOP_P_EPS)
+    full = oracle_proxy(name, 1.0)
+    assert kmax == full["kmax"] == ref["kmax"]
+    cnt = got["count"]
+    assert np.all(ref["count_lo"] <= cnt) and np.all(cnt <= ref["count_hi"])
+    Hq, NQB = cnt.shape
+    for h in range(Hq):
+        for I in range(NQB):
+            k = int(cnt[h, I])
+            assert 1 <= k <= full["count"][h, I]
+            assert got["order"][h, I, :k].tolist() == full["order"][h, I, :k].tolist()
+            assert np.all(got["order"][h, I, k:] == -1)
+            assert got["hrm"][h, I, :k].tolist() == full["hrm"][h, I, :k].tolist()
+            assert not got["hrm"][h, I, k:].any()
+            assert got["n_hrm"][h, I] == int(full["hrm"][h, I, :k].sum())
+    if p == 1.0:
+        assert np.array_equal(cnt, full["count"])
+    print(name, p, "exact", float((cnt == ref["count"]).mean()), "mean k", float(cnt.mean()))
+
+
+@pytest.mark.parametrize("name,p,tau", [("ragged_b128_p64", 0.95, 1e-3), ("qwen_mix", 0.9, 1e-4)])
+def test_attn_on_top_p_lists_matches_oracle(name, p, tau):
+    """The OSK over the (long) lists of the Top-p rule, the oracle's lists given to both sides."""
+    w, d = workload(name), device(name)
+    ref = kap.kap_proxy_top_p(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, p)
+    ws, _ = cosa.alloc_workspace(d["batch"], 1.0)
+    sel = {"order": torch.from_numpy(ref["order"]).cuda(), "count": torch.from_numpy(ref["count"]).cuda()}
+    res = gu.run_attn(d, sel, ref["kmax"], tau, ws)
+    o = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, ref["order"],
+                ref["count"], tau)
+    print(name, p, tau, gu.compare_attn(res, o, w, tau, gu.all_units(w)))
