@@ -127,6 +127,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+// Wait for a phase that this CTA's own copies or MMAs complete, before the
+// CTA exits or frees what they write.  Unlike mbar_wait it ignores the abort
+// flag (an aborted CTA must still let its own transfers land), but it gives
+// up after kDrainPolls polls (tens of milliseconds at most; a transfer that
+// was issued lands within microseconds).
+constexpr uint32_t kDrainPolls = 1u << 14;
+
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i <= kDrainPolls; ++i)
+    if (mbar_try_wait(bar, parity, kPollSuspendNs)) return;
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(

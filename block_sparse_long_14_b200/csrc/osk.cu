@@ -61,7 +61,6 @@ constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr int kBQ = 128;          // query rows per tile (TMEM lanes)
 constexpr int kStages = 1;        // K and V slots per CTA (two CTAs share an SM)
-constexpr uint32_t kDrainLimit = 1u << 22;
 constexpr float kRescaleLog2 = 8.0f;  // re-base O when the row max grows by > 2^8
 
 struct Bars {
@@ -326,10 +325,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     // drain: every load this warp started has landed before the CTA exits
     if (lane == 0) {
-      mbar_wait(&bars->q_full, 0, kDrainLimit, abort, nullptr, 0);
+      mbar_drain(&bars->q_full, 0);
       for (int x = 0; x < kStages; ++x) {
-        if (k_armed[x] >= 0) mbar_wait(&bars->k_full[x], k_armed[x] & 1, kDrainLimit, abort, nullptr, 0);
-        if (v_armed[x] >= 0) mbar_wait(&bars->v_full[x], v_armed[x] & 1, kDrainLimit, abort, nullptr, 0);
+        if (k_armed[x] >= 0) mbar_drain(&bars->k_full[x], k_armed[x] & 1);
+        if (v_armed[x] >= 0) mbar_drain(&bars->v_full[x], v_armed[x] & 1);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -386,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
       tc_commit(&bars->mma_drain);
-      mbar_wait(&bars->mma_drain, 0, kDrainLimit, abort, nullptr, 0);
+      mbar_drain(&bars->mma_drain, 0);
     }
     __syncwarp();
   } else {
