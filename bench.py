@@ -261,6 +261,65 @@ def upload(w, device="cuda"):
                 page_table=torch.from_numpy(np.ascontiguousarray(w.page_table)).to(device))
 
 
+TOP_P = 0.95       # the pages' stage-1 p (Qwen3-8B; Llama's is calibrated per context length)
+DELTA = 200.0      # the pages' Llama-3.1-8B delta in tau_s = delta / N
+
+
+def _timed(fn, stream, reps=2):
+    """Device time of fn() on `stream` (ms), after one untimed call."""
+    import torch
+    fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def pages_rules(cosa, batch, d, nqb_rows, tile_flops, stream):
+    """Top-p stage 1 (p = TOP_P) and the length-adaptive tau_s = DELTA / N on the bench layer."""
+    ws, kmax = cosa.alloc_workspace(batch, 1.0)     # a Top-p row may keep every candidate
+    sel = cosa.proxy_top_p(batch, d["q"], d["k_pages"], d["page_table"], TOP_P, kmax, ws)
+    t_proxy = _timed(lambda: cosa.proxy_top_p(batch, d["q"], d["k_pages"], d["page_table"], TOP_P, kmax, ws,
+                                              out=sel), stream)
+    res = cosa.attn_delta(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"], sel["order"], sel["count"],
+                          kmax, DELTA, ws)
+    t_attn = _timed(lambda: cosa.attn_delta(batch, d["q"], d["k_pages"], d["v_pages"], d["page_table"],
+                                            sel["order"], sel["count"], kmax, DELTA, ws, out=res), stream)
+    cosa.check(ws)
+    vis = int(res["visited"].sum().item())
+    sk = int(res["skipped"].sum().item())
+    return {"p": TOP_P, "delta": DELTA, "ms": t_proxy + t_attn, "proxy_ms": t_proxy, "attn_ms": t_attn,
+            "stage1_budget": vis / nqb_rows, "skip_ratio": sk / max(1, vis),
+            "stage2_budget": (vis - sk) / nqb_rows,
+            "attn_tflops_executed": tile_flops * (2 * vis - sk) / (t_attn * 1e-3) / 1e12}
+
+
+def cached_prefix(cosa, w, d, budget, stream):
+    """The bench layer with its first half as a cached prefix (q_len = kv_len / 2 per sequence)."""
+    q_lens = [L - L // 2 for L in w.seqlens]
+    rows, tok0 = [], 0
+    for L, Lq in zip(w.seqlens, q_lens):
+        rows.append(d["q"][tok0 + L - Lq:tok0 + L])
+        tok0 += L
+    import torch
+    q = rows[0] if len(rows) == 1 else torch.cat(rows)
+    batch = cosa.Batch(w.seqlens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.page_size,
+                       w.num_pages, w.max_pages_per_seq, device="cuda", q_lens=q_lens)
+    ws, kmax = cosa.alloc_workspace(batch, budget)
+    sel = cosa.proxy(batch, q, d["k_pages"], d["page_table"], budget, kmax, ws)
+    t_proxy = _timed(lambda: cosa.proxy(batch, q, d["k_pages"], d["page_table"], budget, kmax, ws, out=sel), stream)
+    res = cosa.attn(batch, q, d["k_pages"], d["v_pages"], d["page_table"], sel["order"], sel["count"], kmax, TAU, ws)
+    t_attn = _timed(lambda: cosa.attn(batch, q, d["k_pages"], d["v_pages"], d["page_table"], sel["order"],
+                                      sel["count"], kmax, TAU, ws, out=res), stream)
+    cosa.check(ws)
+    return {"q_tokens": sum(q_lens), "kv_tokens": sum(w.seqlens), "budget": budget, "tau": TAU,
+            "ms": t_proxy + t_attn, "proxy_ms": t_proxy, "attn_ms": t_attn,
+            "skip_ratio": int(res["skipped"].sum().item()) / max(1, int(res["visited"].sum().item()))}
+
+
 def run_cosa(args, rank, world, local_rank):
     import torch
     import block_sparse_long_14_b200 as cosa
@@ -481,6 +540,20 @@ def run_cosa(args, rank, world, local_rank):
         d2h = h_out.nbytes + h_vis.nbytes + h_skp.nbytes
         e2e = {"value": el / k2 / world, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": k2}
+
+    if rank == 0 and world == 1 and not args.quick:
+        # Informational legs, run after every number the headline line needs: the
+        # pages' own stage rules on the same layer (Top-p stage 1, tau_s = delta / N),
+        # and the layer as prefill after a cached prefix (its first half has keys and
+        # values but no queries).
+        try:
+            extra["pages_rules"] = pages_rules(cosa, batch, d, nqb_rows, tile_flops, stream)
+        except Exception as exc:
+            extra["pages_rules"] = {"error": str(exc)[:200]}
+        try:
+            extra["cached_prefix"] = cached_prefix(cosa, w, d, budget, stream)
+        except Exception as exc:
+            extra["cached_prefix"] = {"error": str(exc)[:200]}
 
     if rank != 0:
         return
