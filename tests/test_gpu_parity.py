@@ -332,3 +332,38 @@ def test_attn_on_top_p_lists_matches_oracle(name, p, tau):
     o = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, ref["order"],
                 ref["count"], tau)
     print(name, p, tau, gu.compare_attn(res, o, w, tau, gu.all_units(w)))
+
+
+def _zero_blocks_workload():
+    """Random Q/K/V (700 tokens, b = 128) with key block 1 all zero (scale 0),
+    one all-zero 16-row query sub-row in q-block 2 and q-block 4 all zero
+    (every score 0: ties broken by the lowest block index)."""
+    from synth import from_arrays
+    rng = np.random.default_rng(31)
+    L = 700
+    q = rng.standard_normal((L, 4, 128)).astype(np.float32)
+    k = rng.standard_normal((L, 2, 128)).astype(np.float32)
+    v = rng.standard_normal((L, 2, 128)).astype(np.float32)
+    k[128:256] = 0.0
+    q[288:304] = 0.0
+    q[512:640] = 0.0
+    return from_arrays([q], [k], [v], 128, 64, shuffle=True, seed=31)
+
+
+@pytest.mark.parametrize("budget,tau", [(0.25, 1e-3), (0.001, 1e-4)])
+def test_zero_blocks_and_single_entry_lists(budget, tau):
+    """Edge cases: an all-zero key block and zero query vectors (quantised to
+    zero with scale 0), and budget 0.1 %, where every list holds one entry (kmax = 1)."""
+    w = _zero_blocks_workload()
+    d = gu.upload(w)
+    got, kmax, ws = gu.run_proxy(d, budget)
+    ref = kap.kap_proxy(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, budget)
+    assert kmax == ref["kmax"]
+    if budget == 0.001:
+        assert kmax == 1
+    gu.assert_proxy_equal(got, ref)
+    sel = {k: torch.from_numpy(v).cuda() for k, v in got.items()}
+    res = gu.run_attn(d, sel, kmax, tau, ws)
+    o = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, ref["order"],
+                ref["count"], tau)
+    print(budget, tau, gu.compare_attn(res, o, w, tau, gu.all_units(w)))
