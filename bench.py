@@ -104,6 +104,25 @@ def rank_seed(cfg, rank, world):
     return None if world == 1 else cfg * 1000 + rank
 
 
+def head_shard(w, rank, world):
+    """Rank `rank`'s share of one layer split by kv head: a contiguous range of
+    Hkv / world kv heads (their pages) and the G query heads of each (their
+    queries).  Every (head, q-block) tile is independent, so the shards need no
+    exchange, and the output stays head-sharded."""
+    import dataclasses
+    if w.num_kv_heads % world:
+        raise ValueError(f"{w.num_kv_heads} kv heads do not split over {world} ranks")
+    nkv = w.num_kv_heads // world
+    G = w.num_q_heads // w.num_kv_heads
+    kv0 = rank * nkv
+    return dataclasses.replace(
+        w, name=f"{w.name}[kv {kv0}..{kv0 + nkv - 1}]", num_q_heads=nkv * G, num_kv_heads=nkv,
+        q=np.ascontiguousarray(w.q[:, kv0 * G:(kv0 + nkv) * G]),
+        k_pages=np.ascontiguousarray(w.k_pages[:, kv0:kv0 + nkv]),
+        v_pages=np.ascontiguousarray(w.v_pages[:, kv0:kv0 + nkv]),
+        meta={**w.meta, "kv_heads": (kv0, kv0 + nkv)})
+
+
 def max_over_ranks(value, dist=None, device="cuda"):
     """Max of a per-rank duration over all ranks (the job's time)."""
     if dist is None:
@@ -330,7 +349,10 @@ def run_cosa(args, rank, world, local_rank):
     if world > 1:
         import torch.distributed as dist
 
-    w = make_workload(args.config, seed=rank_seed(args.config, rank, world))
+    if args.shard == "heads":
+        w = head_shard(make_workload(args.config), rank, world)   # one layer, split by kv head
+    else:
+        w = make_workload(args.config, seed=rank_seed(args.config, rank, world))
     d = upload(w)
     batch = d["batch"]
     budget = w.budgets[0]
@@ -382,7 +404,9 @@ def run_cosa(args, rank, world, local_rank):
     t_attn = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     elapsed = max_over_ranks(elapsed, dist)
     ms_per_step = elapsed / args.steps
-    value = ms_per_step / world          # layers of all ranks run concurrently
+    # ms per layer: the ranks' independent layers run concurrently, or one layer is split
+    per_layer = world if args.shard == "layers" else 1
+    value = ms_per_step / per_layer
 
     # ---- work accounting (identical every step)
     visited = int(res["visited"].sum().item())
@@ -538,7 +562,7 @@ def run_cosa(args, rank, world, local_rank):
         cosa.check(ws)
         h2d = h_q.nbytes + h_k.nbytes + h_v.nbytes + h_t.nbytes
         d2h = h_out.nbytes + h_vis.nbytes + h_skp.nbytes
-        e2e = {"value": el / k2 / world, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+        e2e = {"value": el / k2 / per_layer, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": k2}
 
     if rank == 0 and world == 1 and not args.quick:
@@ -560,11 +584,13 @@ def run_cosa(args, rank, world, local_rank):
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "ms", "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": False,
+        "scaling": "weak" if args.shard == "layers" else "strong",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "cosa",
-        "config": {**workload_config(w), "parallelism": f"independent layers x{world}" if world > 1 else "single"},
+        "config": {**workload_config(w), "parallelism": "single" if world == 1 else
+                   (f"independent layers x{world}" if args.shard == "layers" else f"kv-head shards x{world}")},
         "breakdown_ms": {"proxy": t_proxy, "attn": t_attn},
-        "effective_tflops": dflops / (ms_per_step * 1e-3) / 1e12,
+        "effective_tflops": world * dflops / (ms_per_step * 1e-3) / 1e12,   # all ranks' work
         "attn_executed_tflops": attn_tflops,
         "pct_tc_peak": attn_tflops / pk["bf16_sustained"],
         "proxy_gbs": proxy_gbs,
@@ -603,6 +629,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the tau sweep, dense reference and e2e legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=16384)
+    ap.add_argument("--shard", default="layers", choices=["layers", "heads"],
+                    help="N > 1: each rank its own layer (weak scaling) or one layer split by kv head (strong)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
