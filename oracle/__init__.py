@@ -22,6 +22,8 @@ open points fixed as stated in each function.
   dense    -- brute-force dense causal softmax attention, fp64 (§3.1), used as
               the closed form the OSK oracle must reduce to at budget 100% and
               tau = 0.
+  parallel -- OraclePool: osk tiles evaluated in spawned worker processes
+              (tiles are independent; the pool only distributes them).
   _layout  -- which q-blocks exist and where their rows sit in the packed Q,
               for full prefill and for prefill after a cached prefix
               (q_len < kv_len; a reading, the pages treat full prefill only).

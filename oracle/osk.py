@@ -73,19 +73,55 @@ def osk_tile(qrows, qpos, blocks, order, tau, scale):
 
 
 class PagedSequence:
-    """Logical fp64 view of one sequence's K/V in the page pool (oracle's own gather)."""
+    """Logical fp64 view of one sequence's K/V for one kv head in the page pool (oracle's own gather)."""
 
-    def __init__(self, k_pages_bits, v_pages_bits, table_row, length, block_size):
-        self.k = f32(gather_tokens(k_pages_bits, table_row, length)).astype(np.float64)
-        self.v = f32(gather_tokens(v_pages_bits, table_row, length)).astype(np.float64)
+    def __init__(self, k_pages_bits, v_pages_bits, table_row, length, block_size, kv_head):
+        self.k = f32(gather_tokens(k_pages_bits[:, kv_head:kv_head + 1], table_row, length)[:, 0]).astype(np.float64)
+        self.v = f32(gather_tokens(v_pages_bits[:, kv_head:kv_head + 1], table_row, length)[:, 0]).astype(np.float64)
         self.length = length
         self.b = block_size
 
-    def block(self, kv_head):
-        def get(j):
-            lo, hi = j * self.b, min(self.length, (j + 1) * self.b)
-            return self.k[lo:hi, kv_head], self.v[lo:hi, kv_head], np.arange(lo, hi)
-        return get
+    def block(self, j):
+        lo, hi = j * self.b, min(self.length, (j + 1) * self.b)
+        return self.k[lo:hi], self.v[lo:hi], np.arange(lo, hi)
+
+
+def osk_units(q_bits, k_pages_bits, v_pages_bits, page_table, seqlens, num_kv_heads, block_size,
+              order, count, tau, units=None, q_lens=None):
+    """OSK tile by tile: yields (h, I, rows, out, skipped, delta) for each (h, I) unit.
+
+    rows: the unit's slice of the packed query rows; out fp64 [rows, d];
+    skipped bool / delta fp64 [count[h, I]] in visit order.  Arguments as in osk().
+    Units are visited grouped by (sequence, kv head), so that one gathered view
+    of a sequence's keys and values serves all of its units.
+    """
+    Tq, Hq, d = q_bits.shape
+    G = Hq // num_kv_heads
+    b = block_size
+    scale = 1.0 / math.sqrt(d)
+    NQB = order.shape[1]
+    layout = query_blocks(seqlens, q_lens, b)
+    taus = list(tau) if np.ndim(tau) else [tau] * len(seqlens)
+    seq_of = np.concatenate([np.full(nb - i0, s) for s, (_, i0, nb, _) in enumerate(layout)])
+    blk0 = np.concatenate([[0], np.cumsum([nb - i0 for _, i0, nb, _ in layout])])
+    if units is None:
+        units = [(h, I) for h in range(Hq) for I in range(NQB)]
+    units = sorted(set((int(h), int(I)) for h, I in units), key=lambda u: (seq_of[u[1]], u[0] // G, u))
+    key, seq = None, None
+    for h, I in units:
+        s = int(seq_of[I])
+        if key != (s, h // G):
+            key = (s, h // G)
+            seq = PagedSequence(k_pages_bits, v_pages_bits, page_table[s], seqlens[s], b, h // G)
+        off, i0, _, tq0 = layout[s]
+        i = i0 + I - blk0[s]
+        L = seqlens[s]
+        r0, r1 = max(off, i * b), min(L, (i + 1) * b)        # absolute positions of the rows
+        rows = slice(tq0 + r0 - off, tq0 + r1 - off)          # their place in the packed Q
+        qrows = f32(q_bits[rows, h]).astype(np.float64)
+        k_i = int(count[h, I])
+        o, sk, de = osk_tile(qrows, np.arange(r0, r1), seq.block, order[h, I, :k_i], taus[s], scale)
+        yield h, I, rows, o, sk, de
 
 
 def osk(q_bits, k_pages_bits, v_pages_bits, page_table, seqlens, num_kv_heads, block_size,
@@ -103,39 +139,15 @@ def osk(q_bits, k_pages_bits, v_pages_bits, page_table, seqlens, num_kv_heads, b
     fp64 [Hq, NQB, kmax] (padding False / NaN).
     """
     Tq, Hq, d = q_bits.shape
-    G = Hq // num_kv_heads
-    b = block_size
-    scale = 1.0 / math.sqrt(d)
-    kmax = order.shape[2]
-    NQB = order.shape[1]
-    layout = query_blocks(seqlens, q_lens, b)
-    taus = list(tau) if np.ndim(tau) else [tau] * len(seqlens)
-    seq_of = np.concatenate([np.full(nb - i0, s) for s, (_, i0, nb, _) in enumerate(layout)])
-    blk0 = np.concatenate([[0], np.cumsum([nb - i0 for _, i0, nb, _ in layout])])
-    if units is None:
-        units = [(h, I) for h in range(Hq) for I in range(NQB)]
-    units = sorted(set((int(h), int(I)) for h, I in units), key=lambda u: (seq_of[u[1]], u))
+    NQB, kmax = order.shape[1], order.shape[2]
     out = np.full((Tq, Hq, d), np.nan)
     visited = np.full((Hq, NQB), -1, dtype=np.int32)
     skipped = np.full((Hq, NQB), -1, dtype=np.int32)
     skip = np.zeros((Hq, NQB, kmax), dtype=bool)
     delta = np.full((Hq, NQB, kmax), np.nan)
-    cache = {}
-    for h, I in units:
-        s = int(seq_of[I])
-        if s not in cache:
-            cache.clear()
-            cache[s] = PagedSequence(k_pages_bits, v_pages_bits, page_table[s], seqlens[s], b)
-        seq = cache[s]
-        off, i0, _, tq0 = layout[s]
-        i = i0 + I - blk0[s]
-        L = seqlens[s]
-        r0, r1 = max(off, i * b), min(L, (i + 1) * b)        # absolute positions of the rows
-        rows = slice(tq0 + r0 - off, tq0 + r1 - off)          # their place in the packed Q
-        qrows = f32(q_bits[rows, h]).astype(np.float64)
-        k_i = int(count[h, I])
-        o, sk, de = osk_tile(qrows, np.arange(r0, r1), seq.block(h // G), order[h, I, :k_i],
-                             taus[s], scale)
+    for h, I, rows, o, sk, de in osk_units(q_bits, k_pages_bits, v_pages_bits, page_table, seqlens, num_kv_heads,
+                                           block_size, order, count, tau, units, q_lens):
+        k_i = len(sk)
         out[rows, h] = o
         visited[h, I] = k_i
         skipped[h, I] = int(sk.sum())
