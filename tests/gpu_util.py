@@ -69,11 +69,37 @@ def assert_proxy_equal(got, ref, rows=None):
                                  f"gpu {g[tuple(bad[0])]} vs oracle {r[tuple(bad[0])]}")
 
 
+def _max_abs_v(w):
+    """max |V| over the page pool, from the bf16 bit patterns (sign bit cleared)."""
+    top = int(np.max(np.asarray(w.v_pages).view(np.uint16) & np.uint16(0x7FFF)))
+    return float(np.array([top << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def _unit_ref(ref, h, I, rows):
+    """(out rows, visited, skip, delta) of one tile, from the oracle's full result
+    dict or from OraclePool.run's per-tile dict."""
+    if isinstance(ref, dict) and "out" in ref:
+        k = int(ref["visited"][h, I])
+        return ref["out"][rows, h], k, ref["skip"][h, I, :k], ref["delta"][h, I, :k]
+    r, o, sk, de = ref[(h, I)]
+    assert (r.start, r.stop) == (rows.start, rows.stop), f"unit ({h},{I}): oracle rows {r} vs {rows}"
+    return o, len(sk), sk, de
+
+
 def compare_attn(res, ref, w, tau, units, q_lens=None):
     """Compare GPU OSK results with the oracle on the given (h, I) units.
 
+    ref: the oracle's result dict (osk.osk) or OraclePool.run's per-tile dict.
     q_lens: per-sequence query counts of prefill after a cached prefix (rows
     and list rows then cover only the queries).
+
+    Skip decisions must match except for blocks whose oracle statistic delta
+    lies within DELTA_WINDOW of ln(tau).  A unit with such a flipped decision is
+    still compared element by element: each flipped block moves a row by at
+    most 2 b tau e^DELTA_WINDOW max|V| (its keys weigh below about tau against
+    the running max, and the row sum is at least 1 in those units), which is
+    added to the unit's max-abs tolerance.  Every unit's skipped count must
+    equal the number of skip bits the kernel itself set.
     Returns a dict of statistics; raises AssertionError on a violation.
     """
     out = res["out"].float().cpu().numpy()
@@ -89,37 +115,48 @@ def compare_attn(res, ref, w, tau, units, q_lens=None):
         seq_of += [s] * nq[-1]
         tok0.append(tok0[-1] + Lq)
     blk0 = np.concatenate([[0], np.cumsum(nq)])
-    errs, n_el, max_err, exempt_units, n_skip = 0.0, 0, 0.0, 0, 0
+    errs, n_el, max_err, exempt_units, n_skip, n_flip_total = 0.0, 0, 0.0, 0, 0, 0
+    exempt_max, vmax = 0.0, None
     for h, I in units:
         s = seq_of[I]
         L = w.seqlens[s]
         off = L - q_lens[s]
         i = I - blk0[s] + off // b
-        k = int(ref["visited"][h, I])
+        rows = slice(tok0[s] + max(off, i * b) - off, tok0[s] + min(L, (i + 1) * b) - off)
+        ref_out, k, ref_skip, ref_delta = _unit_ref(ref, h, I, rows)
         assert visited[h, I] == k, f"visited[{h},{I}] {visited[h, I]} != {k}"
-        gs, rs = skipbits[h, I, :k], ref["skip"][h, I, :k]
+        gs = skipbits[h, I, :k]
         assert not skipbits[h, I, k:].any()
-        diff = gs != rs
-        if diff.any():
-            dl = ref["delta"][h, I, :k][diff]
+        assert skipped[h, I] == int(gs.sum()), f"skipped[{h},{I}] {skipped[h, I]} != {int(gs.sum())} skip bits"
+        diff = gs != ref_skip
+        n_flip = int(diff.sum())
+        if n_flip:
+            dl = ref_delta[diff]
             assert np.all(np.abs(dl - log_tau) <= DELTA_WINDOW), (
                 f"unit ({h},{I}): skip decisions differ at {np.flatnonzero(diff).tolist()} with oracle delta "
                 f"{dl.tolist()} vs ln tau {log_tau}")
             exempt_units += 1
-            continue
-        assert skipped[h, I] == int(gs.sum())
+            n_flip_total += n_flip
         n_skip += int(gs.sum())
-        rows = slice(tok0[s] + max(off, i * b) - off, tok0[s] + min(L, (i + 1) * b) - off)
-        e = np.abs(out[rows, h].astype(np.float64) - ref["out"][rows, h])
-        assert np.isfinite(out[rows, h]).all()
-        max_err = max(max_err, float(e.max()))
+        got = out[rows, h]
+        assert np.isfinite(got).all(), f"unit ({h},{I}): non-finite output"
+        e = np.abs(got.astype(np.float64) - ref_out)
+        if n_flip:
+            if vmax is None:
+                vmax = _max_abs_v(w)
+            allow = MAX_ABS + n_flip * 2.0 * b * tau * math.exp(DELTA_WINDOW) * vmax
+            assert e.max() <= allow, f"unit ({h},{I}): max-abs {e.max()} above {allow} with {n_flip} flipped blocks"
+            exempt_max = max(exempt_max, float(e.max()))
+        else:
+            max_err = max(max_err, float(e.max()))
         errs += float(e.sum())
         n_el += e.size
     assert exempt_units <= max(1, len(units) // 100), f"{exempt_units} units with exempt skip differences"
     mean = errs / max(1, n_el)
     assert max_err <= MAX_ABS, f"max-abs {max_err}"
     assert mean <= MEAN_ABS, f"mean-abs {mean}"
-    return dict(max_abs=max_err, mean_abs=mean, units=len(units), exempt_units=exempt_units, skipped=n_skip)
+    return dict(max_abs=max_err, mean_abs=mean, units=len(units), exempt_units=exempt_units,
+                flipped_blocks=n_flip_total, exempt_max_abs=exempt_max, skipped=n_skip)
 
 
 def all_units(w):
@@ -128,15 +165,18 @@ def all_units(w):
 
 
 def sample_units(w, n, seed=0):
-    """A seeded sample of (h, I) tiles that always includes each sequence's first and last q-block."""
+    """A seeded sample of n (h, I) tiles that always includes each sequence's first
+    and last q-block (for every head when n allows)."""
     rng = np.random.default_rng(seed)
     b = w.block_size
     nqb = [(L + b - 1) // b for L in w.seqlens]
     blk0 = np.concatenate([[0], np.cumsum(nqb)])
+    edges = sorted({int(I) for s in range(len(w.seqlens)) for I in (blk0[s], blk0[s + 1] - 1)})
     units = set()
-    for s in range(len(w.seqlens)):
-        for I in (blk0[s], blk0[s + 1] - 1):
-            units.add((int(rng.integers(w.num_q_heads)), int(I)))
+    if len(edges) * w.num_q_heads <= n:
+        units.update((h, I) for I in edges for h in range(w.num_q_heads))
+    else:
+        units.update((int(rng.integers(w.num_q_heads)), I) for I in edges)
     total = int(blk0[-1])
     while len(units) < n:
         units.add((int(rng.integers(w.num_q_heads)), int(rng.integers(total))))
