@@ -191,3 +191,30 @@ def test_proxy_top_p_arguments(lib):
                               None, None, 0, None)
     assert rc == 1
     assert _ws(sh, 1.0)[1] == n_all         # budget 1.0 reports the kmax Top-p needs
+
+
+def test_noalloc_scratch_boundary(lib):
+    """cosa_proxy_noalloc keeps the pooled keys (Hkv x NKB x d int8, rounded up to
+    256 bytes) and their scales (Hkv x NKB fp32) in its fixed array: 8 kv heads
+    at d = 128 take 1,056 bytes per key block, so 3,971 key blocks fit in
+    COSA_NOALLOC_SCRATCH_BYTES and 3,972 are refused with COSA_ERR_WORKSPACE
+    before anything reaches the device."""
+    import torch
+    limit = 4 << 20
+
+    def need(nkb):
+        return (8 * nkb * 128 + 255) // 256 * 256 + 8 * nkb * 4
+
+    assert need(3971) <= limit < need(3972)
+    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced on the refusing path
+
+    def call(nkb):
+        L = nkb * 128
+        sh = _shape(total_tokens=L, total_qblocks=nkb, max_seqlen=L, num_pages=nkb * 2, max_pages_per_seq=nkb * 2)
+        return lib.cosa_proxy_noalloc(ctypes.byref(sh), fake, fake, fake, ctypes.c_float(0.05), 256, fake, fake,
+                                      fake, fake, None)
+
+    assert call(3972) == 3
+    if not torch.cuda.is_available():
+        # without a device the accepted size fails later, at the device query, never at the size check
+        assert call(3971) not in (0, 3)
