@@ -248,6 +248,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 16 consecutive 32-bit columns of this thread's TMEM lane, as raw words.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 // 16 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -315,6 +325,22 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 2^k, exactly, for an integer-valued k <= 0; 0 below the normal range (and for -inf).
+__device__ __forceinline__ float pow2_int(float k) {
+  return k < -126.0f ? 0.0f : __int_as_float((127 + static_cast<int>(k)) << 23);
+}
+
+// The two bf16 values of a packed pair, as fp32 (exact).
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t p) {
+  return make_float2(__uint_as_float(p << 16), __uint_as_float(p & 0xFFFF0000u));
+}
+
+// A packed bf16 pair multiplied by f (fp32 products, rounded back to bf16).
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t p, float f) {
+  const float lo = __uint_as_float(p << 16), hi = __uint_as_float(p & 0xFFFF0000u);
+  return pack_bf16x2(lo * f, hi * f);
 }
 
 }  // namespace cosa

@@ -79,6 +79,7 @@ struct Bars {
   float half_max[2][2][kBQ];   // [c & 1][half][row]: exchange of half-row maxima; the
                                // epilogue reuses the slot after the last computed block
                                // for the partial row sums
+  float half_ref[2][2][kBQ];   // [c & 1][half][row]: exchange of the halves' P references
 };
 
 template <int D, int BK>
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     mbar_init(&bars->s_full[0], 1);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&bars->p_full[x], kSoftmaxThreads);
+      mbar_init(&bars->p_full[x], kSoftmaxWarps);   // one arrival per softmax warp
       mbar_init(&bars->o_done[x], 1);
     }
     mbar_init(&bars->mma_drain, 1);
@@ -413,10 +414,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t s_cols = lane_base + col0;
       bool ok = mbar_wait(&bars->s_full[0], sb, a.wait_limit, abort, a.status, 0x30);
       ok = __all_sync(0xffffffffu, ok) && !aborted;
-      // first pass: the half-row max, 32 columns at a time
+      // One pass over this thread's S columns, 32 at a time: causal mask, half-row
+      // max, and P = exp2(s * log2e/sqrt(d) - tr) in bf16 written back over the
+      // columns already read, with the partial row sum of the bf16-rounded values
+      // (the same P that P V reads, so a dominant key's rounding cancels in O / l).
+      // tr is the thread's reference: the row's running reference mref, raised to
+      // the next integer above a chunk's max when that max exceeds it by more than
+      // 2^8 (the P already written for earlier chunks is then re-based).  References
+      // are integers, so every re-basing multiplies by an exact power of two.
       float mx = -INFINITY;
+      float tr = mref;
+      float2 ls = make_float2(0.0f, 0.0f);
       if (ok) {
         tc_fence_after();
+        const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
         for (int c = 0; c < C::HALF / 32; ++c) {
           float sc[32];
@@ -438,15 +449,49 @@ __global__ void __launch_bounds__(kThreads, 2)
             mx2 = fmaxf(mx2, sc[k + 2]);
             mx3 = fmaxf(mx3, sc[k + 3]);
           }
-          mx = fmaxf(mx, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+          const float cmx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+          mx = fmaxf(mx, cmx);
+          const float cm2 = cmx * sl2;   // -inf for a fully masked chunk
+          const bool raise = cm2 > tr + kRescaleLog2;
+          if (c > 0 && __any_sync(0xffffffffu, raise && tr != -INFINITY)) {
+            // re-base the P of the earlier chunks (rare after a row's first kept block)
+            const float f = raise ? pow2_int(tr - ceilf(cm2)) : 1.0f;
+            tc_wait_st();
+#pragma unroll 1
+            for (int cc = 0; cc < c; ++cc) {
+              uint32_t pk[16];
+              tmem_ld16(s_cols + cc * 16, pk);
+              tc_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pk[e] = scale_bf16x2(pk[e], f);
+              tmem_st16(s_cols + cc * 16, pk);
+            }
+            ls.x *= f;
+            ls.y *= f;
+          }
+          if (raise) tr = ceilf(cm2);
+          const float nb = (tr == -INFINITY) ? 0.0f : -tr;
+          const float2 nbx2 = make_float2(nb, nb);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            // two logits per packed fp32 FMA, two sums per packed add
+            const float2 x = fma_f32x2(make_float2(sc[2 * e], sc[2 * e + 1]), sl2x2, nbx2);
+            pk[e] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+            ls = add_f32x2(ls, unpack_bf16x2(pk[e]));
+          }
+          // P of chunk c goes to columns [16c, 16c + 16) of this thread's half, all already read
+          tmem_st16(s_cols + c * 16, pk);
         }
       }
+      // the skip vote takes the exact running max m; rows past the sequence end vote to skip
       const float m_half = (row_valid && mx != -INFINITY) ? mx * sl2 : -INFINITY;
       const float gap = (m_half == -INFINITY) ? -INFINITY : m_half - m;
       const bool votes_skip = !row_valid || gap < log2_tau;
       const bool wskip = __all_sync(0xffffffffu, votes_skip);
       if (lane == 0) bars->vote[sb][warp] = (ok ? 0 : 2) | (wskip ? 1 : 0);
       bars->half_max[sb][half][r] = m_half;
+      bars->half_ref[sb][half][r] = tr;
       named_bar_sync(1, kSoftmaxThreads);
       int vor = 0, vand = 1;
 #pragma unroll
@@ -462,62 +507,42 @@ __global__ void __launch_bounds__(kThreads, 2)
           ++nskip;
           if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 1;
         }
+        // the dead P stores land before the S buffer is handed back
+        tc_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[sb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
         continue;
       }
       const float m_row = fmaxf(m_half, bars->half_max[sb][half ^ 1][r]);
       const float m_new = fmaxf(m, m_row);
-      // the reference max of P / l / O: re-based lazily (identical in both halves of a row)
-      float new_ref = mref;
-      bool rescale = false;
-      if (n_pv == 0) {
-        if (row_valid) new_ref = m_new;
-      } else {
-        const bool need = row_valid && (m_new > mref + kRescaleLog2);
-        rescale = __any_sync(0xffffffffu, need);
-        if (rescale && row_valid) new_ref = m_new;
-      }
-      // P = exp2(s * log2e/sqrt(d) - ref) in bf16; partial row sum of the fp32 values.
-      // Rows past the sequence end need no masking here: a row of P only feeds the
-      // same row of O, and those rows of O are never written out.
-      float2 ls = make_float2(0.0f, 0.0f);
-      const float nb = (new_ref == -INFINITY) ? 0.0f : -new_ref;
-      const float2 sl2x2 = make_float2(sl2, sl2), nbx2 = make_float2(nb, nb);
-      // second pass over the S columns, 32 at a time (registers are capped at 96 with two
-      // CTAs per SM): P of chunk c goes to columns [16c, 16c + 16) of this thread's
-      // half, all already read
+      // the row's reference: the higher of its two halves' (identical in both threads of the row)
+      const float ref_row = fmaxf(tr, bars->half_ref[sb][half ^ 1][r]);
+      if (__any_sync(0xffffffffu, tr < ref_row)) {
+        // this half's P is re-based to the row's reference (the other half raised it higher)
+        const float f = (tr < ref_row) ? pow2_int(tr - ref_row) : 1.0f;
+        tc_wait_st();
+#pragma unroll 1
+        for (int c = 0; c < C::HALF / 32; ++c) {
+          uint32_t pk[16];
+          tmem_ld16(s_cols + c * 16, pk);
+          tc_wait_ld();
 #pragma unroll
-      for (int c = 0; c < C::HALF / 32; ++c) {
-        float sc[32];
-        tmem_ld32(s_cols + c * 32, sc);
-        tc_wait_ld();
-        if (j >= i) {
-          const int lim = r - (j - i) * b - col0 - c * 32;
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (k > lim) sc[k] = -INFINITY;
+          for (int e = 0; e < 16; ++e) pk[e] = scale_bf16x2(pk[e], f);
+          tmem_st16(s_cols + c * 16, pk);
         }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          // two logits per packed fp32 FMA, two sums per packed add
-          const float2 x = fma_f32x2(make_float2(sc[2 * e], sc[2 * e + 1]), sl2x2, nbx2);
-          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          pk[e] = pack_bf16x2(pv.x, pv.y);
-          ls = add_f32x2(ls, pv);
-        }
-        tmem_st16(s_cols + c * 16, pk);
+        ls.x *= f;
+        ls.y *= f;
       }
-      const float ls0 = ls.x, ls1 = ls.y;
-      if (rescale) {
+      // O and l follow the row's reference (ref_row >= mref: tr starts at mref and only rises)
+      float alpha = 1.0f;
+      if (n_pv > 0 && __any_sync(0xffffffffu, ref_row > mref)) {
         // O must be complete up to the last kept block before it is re-based
         bool okw = mbar_wait(&bars->o_done[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status,
                              0x31);
         if (!__all_sync(0xffffffffu, okw)) { aborted = true; continue; }
         tc_fence_after();
-        const float alpha = row_valid ? ex2_approx(mref - new_ref) : 1.0f;
-        l *= alpha;
+        alpha = pow2_int(mref - ref_row);   // 0 while mref is -inf
 #pragma unroll 1
         for (int c = 0; c < D / 64; ++c) {
           float ov[32];
@@ -529,16 +554,17 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_st32(addr, ov);
         }
       }
-      mref = new_ref;
+      mref = ref_row;
       m = m_new;
-      l += ls0 + ls1;
+      l = l * alpha + (ls.x + ls.y);
       tc_wait_st();
       tc_fence_before();
       if (tid == 0) {
         bars->skip_flag[sb] = 0;
         if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 0;
       }
-      mbar_arrive(&bars->p_full[sb]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[sb]);
       ++n_pv;
     }
     // ---- epilogue: O / l -> bf16

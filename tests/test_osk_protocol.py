@@ -4,7 +4,7 @@ The kernel's producer warp (K and V copies into one slot each), MMA warp
 (S = Q K^T into one TMEM buffer, P V into O) and softmax warps (reading S,
 writing P in place, voting on the skip) hand work to each other through
 mbarriers: q_full; k_full / k_empty and v_full / v_empty for the two slots;
-s_full for S; p_full[2] (all softmax threads arrive) for P and the skip flag;
+s_full for S; p_full[2] (one arrival per softmax warp) for P and the skip flag;
 o_done[2] for P V; and the MMA drain.  This model replays each role's waits
 (with the kernel's parities) and arrivals, with copies and MMAs completing
 asynchronously (MMAs in issue order), for random keep masks and skip
@@ -41,7 +41,7 @@ def run(keep, skip, rescale, rng):
     n_comp = sum(keep)
     q_full, k_full, k_empty, v_full, v_empty = Bar(1), Bar(1), Bar(1), Bar(1), Bar(1)
     s_full, drain = Bar(1), Bar(1)
-    p_full = [Bar(1), Bar(1)]          # the softmax threads arrive together: one arrival here
+    p_full = [Bar(1), Bar(1)]          # the softmax warps arrive together: one arrival here
     o_done = [Bar(1), Bar(1)]
     pending = []                       # async completions, ('copy', bar) or ('mma', [bars])
     armed = {"k": -1, "v": -1}
