@@ -129,15 +129,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map with 128-byte swizzle and 128-byte inner boxes (bf16 unless stated).
+// Tiled tensor map (bf16 and 128-byte swizzle with 128-byte inner boxes unless stated).
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
-              const cuuint32_t* box, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+              const cuuint32_t* box, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint32_t elem[3] = {1, 1, 1};
   std::memset(m, 0, sizeof(*m));
   return fn(m, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
-            strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            strides_bytes, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

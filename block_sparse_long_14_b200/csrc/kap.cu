@@ -32,10 +32,9 @@
 
 #include "cosa_device.cuh"
 #include "cosa_internal.h"
+#include "kap_common.cuh"
 
 namespace cosa {
-
-static constexpr float kTiny = 1.17549435e-38f;  // 2^-126: smallest normal fp32
 
 // ============================================================================ kpool
 template <int D, bool NHD>
@@ -130,23 +129,6 @@ __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, ui
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Sort key: bit 63 = not HRM, bits 31..62 = score mapped to an unsigned
-// order that is descending in the score, bits 0..30 = block index.
-// Ascending keys give (HRM first, score descending, index ascending).
-__device__ __forceinline__ uint64_t make_key(float sc, int j) {
-  uint32_t u = __float_as_uint(sc);
-  if ((u & 0x7FFFFFFFu) == 0) u = 0;                         // -0 -> +0
-  const uint32_t asc = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return (1ull << 63) | (static_cast<uint64_t>(~asc) << 31) | static_cast<uint32_t>(j);
-}
-
-// The score a sort key was made from (make_key is a bijection on non-zero
-// floats and maps both zeros to +0).
-__device__ __forceinline__ float score_of_key(uint64_t key) {
-  const uint32_t asc = ~static_cast<uint32_t>(key >> 31);
-  return __uint_as_float((asc & 0x80000000u) ? (asc & 0x7FFFFFFFu) : ~asc);
-}
-
 __device__ __forceinline__ bool better(float s2, int j2, float s1, int j1) {
   return s2 > s1 || (s2 == s1 && j2 < j1);
 }
@@ -175,40 +157,9 @@ __device__ void bitonic_sort(uint64_t* base, int nseg, int size, int stride) {
   }
 }
 
-// Tile of the proxy: (q-block I, GT query heads h0.. sharing kv head kv).
-// Its query rows are the tile rows [rlo, rhi) (absolute positions i*b + r);
-// rlo > 0 only in the first q-block after a cached prefix.  Row r of the
-// tile is packed q row q_row0 + i*b + r.  kb0: key block 0 of the sequence
-// in the pooled-key arrays.  bad: the offsets disagree with the lengths.
-struct Tile {
-  int I, h0, kv, s, kb0, i, L, rlo, rhi, n, npow2;
-  long q_row0;
-  bool bad;
-};
-
-// Sub-row v (tile rows 16v .. 16v + 15) holds at least one query row.
-__device__ __forceinline__ bool sub_present(const Tile& t, int v) { return v * 16 < t.rhi && v * 16 + 16 > t.rlo; }
-
 template <int GT>
 __device__ __forceinline__ Tile tile_of(const ScoreArgs& a) {
-  Tile t;
-  const int ngroups = a.num_q_heads / GT;
-  t.I = a.nqb_total - 1 - static_cast<int>(blockIdx.x) / ngroups;   // longest rows first
-  t.h0 = (static_cast<int>(blockIdx.x) % ngroups) * GT;
-  t.kv = t.h0 / (a.num_q_heads / a.num_kv_heads);
-  t.s = find_seq(a.cu_qblocks, a.batch, t.I);
-  const SeqSpan sp = seq_span(a.cu_seqlens, a.kv_lens, t.s, a.block_size);
-  t.kb0 = __ldg(a.cu_kblocks + t.s);
-  t.i = t.I - __ldg(a.cu_qblocks + t.s) + sp.i0;
-  t.L = sp.L;
-  t.q_row0 = sp.q_row0;
-  t.rlo = max(0, sp.off - t.i * a.block_size);
-  t.rhi = min(a.block_size, t.L - t.i * a.block_size);
-  t.bad = sp.off < 0 || t.rlo >= t.rhi;
-  t.n = t.i + 1;
-  t.npow2 = 1;
-  while (t.npow2 < t.n) t.npow2 <<= 1;
-  return t;
+  return tile_at<GT>(a, static_cast<int>(blockIdx.x));
 }
 
 // Pooling of one tile (256 threads): the 16-row sub-row sums (token by token,
@@ -709,17 +660,6 @@ __device__ void select_tile(const ScoreArgs& a, const Tile& tl, const int8_t* am
 }
 
 // ============================================================ tcgen05 scoring
-// D[tmem] (+)= A[smem] * B[smem]^T with tcgen05 kind::i8: s8 x s8 -> exact s32.
-__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // 16 TMEM lanes x 32 columns: thread t receives lane t/4 in registers
 // 4c, 4c+1 and lane t/4 + 8 in registers 4c+2, 4c+3, at columns
 // 8c + 2 (t % 4) + {0, 1}, c = 0..3.
@@ -736,14 +676,6 @@ constexpr int kTcN = 64;                  // candidate key blocks per score tile
 constexpr int kTcRing = 2;                // key tiles in flight
 constexpr int kTcTmemCols = 2 * kTcN;     // two accumulators: 3 CTAs per SM fit in TMEM
 constexpr uint32_t kTcWaitLimit = 1u << 22;
-
-// Instruction descriptor of kind::i8: D format S32 (2) at bit 4, A and B
-// signed 8-bit (1) at bits 7 and 10, K-major operands, N >> 3 at bit 17,
-// M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-         (static_cast<uint32_t>(M >> 4) << 24);
-}
 
 size_t select_tc_smem_bytes(int GT, int npow2_max, int scratch_bytes) {
   return kTcRing * kTcN * 128 + 64 * 128 + static_cast<size_t>(GT) * npow2_max * 8 +
