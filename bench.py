@@ -10,10 +10,13 @@ the timed region starts; the 1.5 GiB of inputs per step exceed the 126 MB L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cosa|reference]
 
-Multi-GPU (torchrun): each rank runs its own layer (independent units, no
-data-path collective); value = total layers / max-over-ranks time.
-The reference arm times the CPU oracle on a bounded sample of the same
-workload and extrapolates to ms per layer.
+Multi-GPU (torchrun): by default one layer is split by kv head across the
+ranks (every (head, q-block) tile is independent, so there is no data-path
+exchange and the output stays head-sharded); value = the layer's
+max-over-ranks time.  --shard layers gives each rank its own layer instead.
+The reference arm times the CPU oracle on the same layer: the proxy on all
+of it, the attention on a seeded sample of its tiles scaled by visited
+blocks to ms per layer (OracleLayer).
 """
 
 from __future__ import annotations
@@ -44,8 +47,21 @@ def peaks():
     if os.path.exists(p):
         d = json.load(open(p))
         return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
-                    source="measured")
-    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+def tensor_peak(pk, clocks):
+    """The dense bf16 peak that matches the clocks sampled in the timed region:
+    the burst figure (a cuBLAS GEMM timed alone, at the maximum SM clock) scaled
+    by the median SM clock under load over that maximum, capped at 1.  A short
+    region runs at the maximum clock, where this is the burst figure itself."""
+    mhz = (clocks or {}).get("sm_mhz")
+    if not mhz:
+        return pk["bf16"], f"{pk['source']} bf16_tflops (burst; no clock samples)"
+    ratio = min(1.0, float(mhz) / float(pk["sm_max_mhz"]))
+    return pk["bf16"] * ratio, (f"{pk['source']} bf16_tflops (burst, {pk['bf16']:.1f}) x median SM clock "
+                                f"{mhz:.0f} / {pk['sm_max_mhz']:.0f} MHz")
 
 
 def measured_traffic():
@@ -214,49 +230,72 @@ class Clocks:
 
 # ------------------------------------------------------------------ CPU side
 
-def oracle_sample(seq_tokens=16384, seed=CONFIG_ID):
-    """Time the oracle (proxy + OSK) on the first `seq_tokens` tokens of the
-    128K layer shape and extrapolate to a full layer by visited blocks."""
-    from oracle import kap, osk
-    from synth import make_custom
-    from synth.workloads import WORKLOADS
-    spec = dict(WORKLOADS[CONFIG_ID])
-    spec.pop("seqlens")
-    spec.pop("name")
-    w = make_custom([seq_tokens], name="llama8b_128k_prefix", seed=seed, **spec)
-    t0 = time.perf_counter()
-    r = kap.kap_proxy(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, BUDGET)
-    o = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, r["order"],
-                r["count"], TAU)
-    dt = time.perf_counter() - t0
-    b = w.block_size
-    nfull = 131072 // b
-    bp = kap.budget_bp(BUDGET)
-    visited_full = w.num_q_heads * sum(kap.keep_count(n, bp) for n in range(1, nfull + 1))
-    visited_sample = int(o["visited"].sum())
-    ms_layer = dt * 1e3 * visited_full / visited_sample
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return ms_layer, dict(kind="oracle", cores=threads,
-                          sample=f"oracle proxy+OSK on the first {seq_tokens} tokens of the 128K layer shape "
-                                 f"(all 32 heads, budget {BUDGET}, tau {TAU}): {dt:.1f} s for {visited_sample} "
-                                 f"visited blocks, scaled to the layer's {visited_full}")
+class OracleLayer:
+    """The oracle (proxy + OSK) on the bench layer, timed on the host's cores.
+
+    The proxy oracle runs on the whole 128K layer in this process (one thread:
+    integer dot products and fp32 sums).  The OSK oracle's tiles are
+    independent; a seeded sample of them, drawn from every q-block of the
+    layer, runs on worker processes (oracle.parallel.OraclePool, one BLAS
+    thread each), and its wall time is scaled to the whole layer by visited
+    blocks (the oracle's cost per tile is one fp64 tile product pair per
+    visited block)."""
+
+    def __init__(self, workers=None):
+        from oracle import kap
+        from oracle.parallel import OraclePool
+        from synth import make_workload
+        self.w = make_workload(CONFIG_ID)
+        w = self.w
+        t0 = time.perf_counter()
+        self.sel = kap.kap_proxy(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, BUDGET)
+        self.proxy_s = time.perf_counter() - t0
+        self.pool = OraclePool(w, workers=workers)
+        self.tiles = [(h, I) for h in range(w.num_q_heads) for I in range(self.sel["count"].shape[1])]
+        self.visited_all = int(self.sel["count"].sum())
+
+    def sample(self, fraction, seed):
+        """(ms per layer estimate, description) from one sample of the OSK tiles."""
+        rng = np.random.default_rng(seed)
+        n = max(1, int(round(fraction * len(self.tiles))))
+        pick = rng.choice(len(self.tiles), size=n, replace=False)
+        units = [self.tiles[x] for x in pick]
+        visited = int(sum(int(self.sel["count"][h, I]) for h, I in units))
+        t0 = time.perf_counter()
+        self.pool.run(self.sel["order"], self.sel["count"], TAU, units)
+        osk_s = time.perf_counter() - t0
+        osk_full = osk_s * self.visited_all / visited
+        ms = (self.proxy_s + osk_full) * 1e3
+        desc = (f"proxy oracle timed on the whole 128K layer ({self.proxy_s:.1f} s, 1 thread); OSK oracle timed on "
+                f"{n} of {len(self.tiles)} (head, q-block) tiles drawn uniformly from the whole layer (seed {seed}): "
+                f"{visited} visited blocks in {osk_s:.1f} s on {self.pool.workers} worker processes (1 BLAS thread "
+                f"each), scaled by visited blocks to the layer's {self.visited_all} ({osk_full:.1f} s); "
+                f"budget {BUDGET}, tau {TAU}")
+        return ms, desc
+
+    def close(self):
+        self.pool.close()
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands, on the host's cores (rank 0 only)."""
     if rank != 0:
         return
-    times = []
-    cb = None
-    for _ in range(args.warmup):
-        pass   # the oracle has no warm-up state; warm-up steps are not run to bound the CPU time
-    for _ in range(args.steps):
-        v, cb = oracle_sample(seq_tokens=args.ref_tokens)
-        times.append(v)
+    layer = OracleLayer()
+    try:
+        for k in range(args.warmup):
+            pass   # the oracle keeps no warm state; warm-up samples are not run, to bound the CPU time
+        times, desc = [], ""
+        for k in range(args.steps):
+            v, desc = layer.sample(args.ref_fraction, seed=1000 + k)
+            times.append(v)
+    finally:
+        layer.close()
     value = statistics.mean(times)
-    cb["value"] = value
-    cb["unit"] = "ms"
+    cb = {"kind": "oracle", "cores": layer.pool.workers, "value": value, "unit": "ms",
+          "sample": f"mean over {args.steps} samples; last: {desc}"}
     line = {"metric": METRIC, "value": value, "unit": "ms", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False, "scaling": "strong",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": "llama8b_128k", "seq_len": 131072, "budget": BUDGET, "tau": TAU},
             "cpu_baseline": cb,
@@ -350,7 +389,9 @@ def run_cosa(args, rank, world, local_rank):
         import torch.distributed as dist
 
     if args.shard == "heads":
-        w = head_shard(make_workload(args.config), rank, world)   # one layer, split by kv head
+        w = make_workload(args.config)
+        if world > 1:
+            w = head_shard(w, rank, world)   # one layer, split by kv head
     else:
         w = make_workload(args.config, seed=rank_seed(args.config, rank, world))
     d = upload(w)
@@ -582,6 +623,7 @@ def run_cosa(args, rank, world, local_rank):
     if rank != 0:
         return
     clocks = clk.summary()
+    tc_peak, tc_peak_source = tensor_peak(pk, clocks)
     line = {
         "metric": METRIC, "value": value, "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": False,
@@ -592,16 +634,16 @@ def run_cosa(args, rank, world, local_rank):
         "breakdown_ms": {"proxy": t_proxy, "attn": t_attn},
         "effective_tflops": world * dflops / (ms_per_step * 1e-3) / 1e12,   # all ranks' work
         "attn_executed_tflops": attn_tflops,
-        "pct_tc_peak": attn_tflops / pk["bf16_sustained"],
+        "pct_tc_peak": attn_tflops / tc_peak,
         "proxy_gbs": proxy_gbs,
         "pct_hbm_proxy": proxy_gbs / pk["hbm_gbs"],
         "realized_budget": {"stage1": visited / nqb_rows, "stage2": (visited - skipped) / nqb_rows,
                             "skip_ratio": skipped / visited},
-        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": attn_tflops / pk["bf16_sustained"],
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / tc_peak,
                      "traffic": measured_traffic() if CONFIG_ID == args.config else None,
                      "kernel": "osk_kernel<128,128>",
-                     "peak_source": f"{pk['source']} bf16_tflops_sustained (kernel timed inside repeated steps)",
+                     "peak_source": tc_peak_source,
                      "algorithmic": f"{exec_flops:.4e} FLOP per launch = 2*128*128*128 * (visited + kept)"},
         "proxy_roofline": {"bound": "hbm", "achieved": proxy_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                            "frac": proxy_gbs / pk["hbm_gbs"], "algorithmic_bytes": proxy_bytes,
@@ -612,10 +654,13 @@ def run_cosa(args, rank, world, local_rank):
         **extra,
     }
     if world == 1 and not args.no_cpu_baseline:
-        v, cb = oracle_sample(seq_tokens=args.ref_tokens)
-        cb["value"] = v
-        cb["unit"] = "ms"
-        line["cpu_baseline"] = cb
+        layer = OracleLayer()
+        try:
+            v, desc = layer.sample(args.ref_fraction, seed=CONFIG_ID)
+        finally:
+            layer.close()
+        line["cpu_baseline"] = {"value": v, "unit": "ms", "cores": layer.pool.workers, "kind": "oracle",
+                                "sample": desc}
     print(json.dumps(line), flush=True)
 
 
@@ -628,9 +673,11 @@ def main():
     ap.add_argument("--config", type=int, default=CONFIG_ID)
     ap.add_argument("--quick", action="store_true", help="skip the tau sweep, dense reference and e2e legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-tokens", type=int, default=16384)
-    ap.add_argument("--shard", default="layers", choices=["layers", "heads"],
-                    help="N > 1: each rank its own layer (weak scaling) or one layer split by kv head (strong)")
+    ap.add_argument("--ref-fraction", type=float, default=0.03,
+                    help="share of the layer's (head, q-block) tiles the oracle's OSK leg times per sample")
+    ap.add_argument("--shard", default="heads", choices=["layers", "heads"],
+                    help="N > 1: one layer split by kv head across the ranks (default; strong scaling, "
+                         "no exchange) or each rank its own layer (weak scaling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "Batch", "CosaError", "PAGES_HND", "PAGES_NHD", "alloc_workspace", "attn", "attn_delta", "attn_masked", "check", "lib", "proxy", "proxy_top_p", "remap",
-    "set_wait_limit", "tau_from_delta", "workspace_size", "LIB_PATH",
+    "set_wait_limit", "workspace_size", "LIB_PATH",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -297,23 +297,6 @@ def attn_masked(batch: Batch, q, k_pages, v_pages, page_table, order, count, kma
     jumping over pages)."""
     return _attn("cosa_attn_masked", batch, q, k_pages, v_pages, page_table, order, count, kmax, tau, workspace,
                  out, skipbits, keep=keep)
-
-
-def tau_from_delta(delta: float, seq_len: int) -> float:
-    """The length-adaptive skip threshold of the paper (§5.1 "Hyperparameters",
-    Appendix D.1 "CoSA settings"; the operating points there are delta = 2000
-    for Qwen3-8B and 200 for Llama-3.1-8B): tau = delta / N with N the
-    sequence length in tokens; delta = -1 turns the in-kernel skip off
-    (tau = 0).  `attn_delta` applies the same mapping on the device, one
-    tau per sequence of a ragged batch."""
-    if delta == -1:
-        return 0.0
-    if not (delta >= 0 and seq_len > 0):
-        raise ValueError(f"delta must be -1 or >= 0 and seq_len > 0 (got {delta}, {seq_len})")
-    tau = float(delta) / float(seq_len)
-    if not tau < 1.0:
-        raise ValueError(f"delta / seq_len = {tau} is not a threshold in [0, 1)")
-    return tau
 
 
 def check(workspace):
