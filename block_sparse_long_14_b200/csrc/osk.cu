@@ -49,19 +49,16 @@
 
 #include "cosa_device.cuh"
 #include "cosa_internal.h"
+#include "osk_common.cuh"
 
 namespace cosa {
 
 namespace {
 
-constexpr int kSoftmaxWarps = 8;
-constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
-constexpr int kBQ = 128;          // query rows per tile (TMEM lanes)
 constexpr int kStages = 1;        // K and V slots per CTA (two CTAs share an SM)
-constexpr float kRescaleLog2 = 8.0f;  // re-base O when the row max grows by > 2^8
 
 struct Bars {
   uint64_t q_full;
@@ -110,34 +107,6 @@ struct Cfg {
   static_assert(OFF_BAR + sizeof(Bars) <= static_cast<size_t>(SMEM), "barrier block inside the allocation");
   static_assert(OFF_BAR % 8 == 0, "mbarrier alignment");
 };
-
-// Copy one key block (K or V) of `nvalid` tokens into a 128B-swizzled stage
-// by hand, zero-filling rows past the sequence end or on a missing page.
-template <int D, int BK>
-__device__ void manual_block_copy(unsigned char* stage, const __nv_bfloat16* pool, const int32_t* pt_row,
-                                  int j, int nvalid, const OskArgs& a, int g, int lane) {
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  const int ppb = a.block_size / a.page_size;
-  for (int idx = lane; idx < BK * CH; idx += 32) {
-    const int row = idx / CH, ch = idx % CH;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (row < nvalid) {
-      const int page = __ldg(pt_row + j * ppb + row / a.page_size);
-      if (page >= 0 && page < a.num_pages) {
-        const long tok = a.nhd ? (static_cast<long>(page) * a.page_size + row % a.page_size) * a.num_kv_heads + g
-                               : (static_cast<long>(page) * a.num_kv_heads + g) * a.page_size + row % a.page_size;
-        const __nv_bfloat16* src = pool + tok * D + ch * 8;
-        v = __ldg(reinterpret_cast<const uint4*>(src));
-      } else {
-        report(a.status, kErrBounds, 0x300);
-      }
-    }
-    const int atom = ch >> 3, cc = ch & 7;
-    *reinterpret_cast<uint4*>(stage + atom * (BK * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
-  }
-  fence_proxy_async();
-  __syncwarp();
-}
 
 }  // namespace
 
@@ -338,27 +307,35 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
       bool ok = mbar_wait(&bars->q_full, 0, a.wait_limit, abort, a.status, 0x20);
       int kept = 0;
-      // S = Q K^T of block t into the S buffer
-      auto issue_s = [&](int t) -> bool {
-        const int slot = t % kStages, use = t / kStages;
+      // S = Q K^T of the u-th computed block into the S buffer (its commits follow separately)
+      auto issue_s = [&](int u) -> bool {
+        const int slot = u % kStages, use = u / kStages;
         if (!mbar_wait(&bars->k_full[slot], use & 1, a.wait_limit, abort, a.status, 0x21)) return false;
         tc_fence_after();
-        const uint32_t d_s = tmem;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t ad = sw128_desc(q_base + (ks >> 2) * (kBQ * 128) + (ks & 3) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(k_base + slot * C::KV_BYTES + (ks >> 2) * (BK * 128) + (ks & 3) * 32, 16, 1024);
-          tc_mma_ss(d_s, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
+          tc_mma_ss(tmem, ad, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&bars->s_full[0]);
-        tc_commit(&bars->k_empty[slot]);
         return true;
       };
-      for (int t = 0, u = 0; t < n && ok; ++t) {
-        if (keep_row != nullptr && __ldg(keep_row + t) == 0) continue;
-        // S of block u takes the buffer whose P V (block u-1) was issued just before
-        ok = issue_s(u);
-        if (!ok) break;
+      auto commit_s = [&](int u) {
+        tc_commit(&bars->s_full[0]);
+        tc_commit(&bars->k_empty[u % kStages]);
+      };
+      // the next list entry at or after x that is computed (every one, unless a keep mask passes some over)
+      auto next_entry = [&](int x) {
+        if (keep_row != nullptr)
+          while (x < n && __ldg(keep_row + x) == 0) ++x;
+        return x;
+      };
+      int t = next_entry(0);
+      if (t < n && ok) {
+        ok = issue_s(0);
+        if (ok) commit_s(0);
+      }
+      for (int u = 0; t < n && ok; ++u) {
         const int vslot = u % kStages, vuse = u / kStages;
         ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, a.wait_limit, abort, a.status, 0x23);
         if (ok) ok = mbar_wait(&bars->v_full[vslot], vuse & 1, a.wait_limit, abort, a.status, 0x24);
@@ -376,13 +353,22 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint64_t bd = sw128_desc(v_base + vslot * C::KV_BYTES + kk * 2048, BK * 128, 1024);
             tc_mma_ts(d_o, a_t, bd, C::IDESC_PV, (kept > 0 || kk > 0) ? 1u : 0u);
           }
+        } else {
+          mbar_arrive(&bars->v_empty[vslot]);   // no MMA reads this V
+        }
+        // S of the next computed block queues right behind P V (the tensor pipe keeps issue
+        // order, so P V has read P before S overwrites it); the commits follow, and each
+        // arrives once every MMA issued before it has completed
+        const int tn = next_entry(t + 1);
+        const bool has_next = tn < n;
+        if (has_next) ok = issue_s(u + 1);
+        if (!skip) {
           tc_commit(&bars->v_empty[vslot]);
           tc_commit(&bars->o_done[kept & 1]);
           ++kept;
-        } else {
-          mbar_arrive(&bars->v_empty[vslot]);
         }
-        ++u;
+        if (has_next && ok) commit_s(u + 1);
+        t = tn;
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
       tc_commit(&bars->mma_drain);
@@ -391,229 +377,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncwarp();
   } else {
     // =========================================================== softmax (warps 0-7)
-    const int quad = warp & 3, half = warp >> 2;
-    const int r = quad * 32 + lane;                 // tile row = TMEM lane
-    const int col0 = half * C::HALF;                // first key column of this thread
-    const bool row_valid = r >= rlo && r < rhi;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const float sl2 = a.scale_log2;
-    float m = -INFINITY, mref = -INFINITY, l = 0.0f;
-    int n_pv = 0, nskip = 0;
-    bool aborted = false;
-    int j_next = __ldg(ord);
-    int ncomp = 0;   // entries computed so far
-    for (int t = 0; t < n; ++t) {
-      const int j = j_next;
-      if (t + 1 < n) j_next = __ldg(ord + t + 1);
-      if (keep_row != nullptr && __ldg(keep_row + t) == 0) {
-        if (tid == 0 && a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 0;
-        continue;
-      }
-      const int sb = ncomp & 1;
-      ++ncomp;
-      const uint32_t s_cols = lane_base + col0;
-      bool ok = mbar_wait(&bars->s_full[0], sb, a.wait_limit, abort, a.status, 0x30);
-      ok = __all_sync(0xffffffffu, ok) && !aborted;
-      // One pass over this thread's S columns, 32 at a time: causal mask, half-row
-      // max, and P = exp2(s * log2e/sqrt(d) - tr) in bf16 written back over the
-      // columns already read, with the partial row sum of the bf16-rounded values
-      // (the same P that P V reads, so a dominant key's rounding cancels in O / l).
-      // tr is the thread's reference: the row's running reference mref, raised to
-      // the next integer above a chunk's max when that max exceeds it by more than
-      // 2^8 (the P already written for earlier chunks is then re-based).  References
-      // are integers, so every re-basing multiplies by an exact power of two.
-      float mx = -INFINITY;
-      float tr = mref;
-      float2 ls = make_float2(0.0f, 0.0f);
-      if (ok) {
-        tc_fence_after();
-        const float2 sl2x2 = make_float2(sl2, sl2);
-#pragma unroll
-        for (int c = 0; c < C::HALF / 32; ++c) {
-          float sc[32];
-          tmem_ld32(s_cols + c * 32, sc);
-          tc_wait_ld();
-          // causal mask (only the diagonal block, or a block past it, can hide keys):
-          // key k of block j is visible to row r iff j*b + k <= i*b + r
-          if (j >= i) {
-            const int lim = r - (j - i) * b - col0 - c * 32;
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (k > lim) sc[k] = -INFINITY;
-          }
-          float mx0 = sc[0], mx1 = sc[1], mx2 = sc[2], mx3 = sc[3];
-#pragma unroll
-          for (int k = 4; k < 32; k += 4) {
-            mx0 = fmaxf(mx0, sc[k]);
-            mx1 = fmaxf(mx1, sc[k + 1]);
-            mx2 = fmaxf(mx2, sc[k + 2]);
-            mx3 = fmaxf(mx3, sc[k + 3]);
-          }
-          const float cmx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-          mx = fmaxf(mx, cmx);
-          const float cm2 = cmx * sl2;   // -inf for a fully masked chunk
-          const bool raise = cm2 > tr + kRescaleLog2;
-          if (c > 0 && __any_sync(0xffffffffu, raise && tr != -INFINITY)) {
-            // re-base the P of the earlier chunks (rare after a row's first kept block)
-            const float f = raise ? pow2_int(tr - ceilf(cm2)) : 1.0f;
-            tc_wait_st();
-#pragma unroll 1
-            for (int cc = 0; cc < c; ++cc) {
-              uint32_t pk[16];
-              tmem_ld16(s_cols + cc * 16, pk);
-              tc_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) pk[e] = scale_bf16x2(pk[e], f);
-              tmem_st16(s_cols + cc * 16, pk);
-            }
-            ls.x *= f;
-            ls.y *= f;
-          }
-          if (raise) tr = ceilf(cm2);
-          const float nb = (tr == -INFINITY) ? 0.0f : -tr;
-          const float2 nbx2 = make_float2(nb, nb);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            // two logits per packed fp32 FMA, two sums per packed add
-            const float2 x = fma_f32x2(make_float2(sc[2 * e], sc[2 * e + 1]), sl2x2, nbx2);
-            pk[e] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
-            ls = add_f32x2(ls, unpack_bf16x2(pk[e]));
-          }
-          // P of chunk c goes to columns [16c, 16c + 16) of this thread's half, all already read
-          tmem_st16(s_cols + c * 16, pk);
-        }
-      }
-      // the skip vote takes the exact running max m; rows past the sequence end vote to skip
-      const float m_half = (row_valid && mx != -INFINITY) ? mx * sl2 : -INFINITY;
-      const float gap = (m_half == -INFINITY) ? -INFINITY : m_half - m;
-      const bool votes_skip = !row_valid || gap < log2_tau;
-      const bool wskip = __all_sync(0xffffffffu, votes_skip);
-      if (lane == 0) bars->vote[sb][warp] = (ok ? 0 : 2) | (wskip ? 1 : 0);
-      bars->half_max[sb][half][r] = m_half;
-      bars->half_ref[sb][half][r] = tr;
-      named_bar_sync(1, kSoftmaxThreads);
-      int vor = 0, vand = 1;
-#pragma unroll
-      for (int w = 0; w < kSoftmaxWarps; ++w) {
-        const int v = bars->vote[sb][w];
-        vor |= v;
-        vand &= v;
-      }
-      if (vor & 2) { aborted = true; break; }
-      if (vand & 1) {
-        if (tid == 0) {
-          bars->skip_flag[sb] = 1;
-          ++nskip;
-          if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 1;
-        }
-        // the dead P stores land before the S buffer is handed back
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
-        continue;
-      }
-      const float m_row = fmaxf(m_half, bars->half_max[sb][half ^ 1][r]);
-      const float m_new = fmaxf(m, m_row);
-      // the row's reference: the higher of its two halves' (identical in both threads of the row)
-      const float ref_row = fmaxf(tr, bars->half_ref[sb][half ^ 1][r]);
-      if (__any_sync(0xffffffffu, tr < ref_row)) {
-        // this half's P is re-based to the row's reference (the other half raised it higher)
-        const float f = (tr < ref_row) ? pow2_int(tr - ref_row) : 1.0f;
-        tc_wait_st();
-#pragma unroll 1
-        for (int c = 0; c < C::HALF / 32; ++c) {
-          uint32_t pk[16];
-          tmem_ld16(s_cols + c * 16, pk);
-          tc_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = scale_bf16x2(pk[e], f);
-          tmem_st16(s_cols + c * 16, pk);
-        }
-        ls.x *= f;
-        ls.y *= f;
-      }
-      // O and l follow the row's reference (ref_row >= mref: tr starts at mref and only rises)
-      float alpha = 1.0f;
-      if (n_pv > 0 && __any_sync(0xffffffffu, ref_row > mref)) {
-        // O must be complete up to the last kept block before it is re-based
-        bool okw = mbar_wait(&bars->o_done[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status,
-                             0x31);
-        if (!__all_sync(0xffffffffu, okw)) { aborted = true; continue; }
-        tc_fence_after();
-        alpha = pow2_int(mref - ref_row);   // 0 while mref is -inf
-#pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {
-          float ov[32];
-          const uint32_t addr = lane_base + C::TMEM_O + half * (D / 2) + c * 32;
-          tmem_ld32(addr, ov);
-          tc_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tmem_st32(addr, ov);
-        }
-      }
-      mref = ref_row;
-      m = m_new;
-      l = l * alpha + (ls.x + ls.y);
-      tc_wait_st();
-      tc_fence_before();
-      if (tid == 0) {
-        bars->skip_flag[sb] = 0;
-        if (a.skipbits != nullptr) a.skipbits[row_id * a.kmax + t] = 0;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[sb]);
-      ++n_pv;
-    }
-    // ---- epilogue: O / l -> bf16
-    bool ok = !aborted && n_pv >= 1;
-    if (ok) ok = mbar_wait(&bars->o_done[(n_pv - 1) & 1], ((n_pv - 1) >> 1) & 1, a.wait_limit, abort, a.status, 0x32);
-    ok = __all_sync(0xffffffffu, ok);
-    float (*half_l)[kBQ] = bars->half_max[ncomp & 1];   // idle since the barrier of the last computed block
-    half_l[half][r] = l;
-    if (lane == 0) bars->vote_end[warp] = ok ? 1 : 0;
-    named_bar_sync(1, kSoftmaxThreads);
-    int all_ok = 1;
-#pragma unroll
-    for (int w = 0; w < kSoftmaxWarps; ++w) all_ok &= bars->vote_end[w];
-    if (ncomp == 0) {
-      // a keep mask that leaves nothing of the row: zero output, like an empty list
-      if (row_valid) {
-        uint4* dst = reinterpret_cast<uint4*>(a.out + ((q_row0 + i * b + r) * a.num_q_heads + h) * D +
-                                              half * (D / 2));
-        for (int q4 = 0; q4 < D / 16; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    } else if (all_ok) {
-      tc_fence_after();
-      const float lrow = half_l[0][r] + half_l[1][r];
-      const float inv_l = (row_valid && lrow > 0.0f) ? 1.0f / lrow : 0.0f;
-      __nv_bfloat16* dst = a.out + ((q_row0 + i * b + r) * a.num_q_heads + h) * D + half * (D / 2);
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        float ov[32];
-        tmem_ld32(lane_base + C::TMEM_O + half * (D / 2) + c * 32, ov);
-        tc_wait_ld();
-        if (row_valid) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 w4;
-            w4.x = pack_bf16x2(ov[q4 * 8 + 0] * inv_l, ov[q4 * 8 + 1] * inv_l);
-            w4.y = pack_bf16x2(ov[q4 * 8 + 2] * inv_l, ov[q4 * 8 + 3] * inv_l);
-            w4.z = pack_bf16x2(ov[q4 * 8 + 4] * inv_l, ov[q4 * 8 + 5] * inv_l);
-            w4.w = pack_bf16x2(ov[q4 * 8 + 6] * inv_l, ov[q4 * 8 + 7] * inv_l);
-            *reinterpret_cast<uint4*>(dst + c * 32 + q4 * 8) = w4;
-          }
-        }
-      }
-    }
-    if (tid == 0) {
-      a.visited[row_id] = ncomp;
-      a.skipped[row_id] = nskip;
-      if (a.skipbits != nullptr)
-        for (int t = n; t < a.kmax; ++t) a.skipbits[row_id * a.kmax + t] = 0;
-    }
+    const SoftmaxTile x{tmem, warp, 1, i, b, rlo, rhi, q_row0, h, row_id, n, ord, keep_row, log2_tau};
+    const SoftmaxSync y{&bars->s_full[0], bars->p_full, bars->o_done, bars->skip_flag, &bars->vote[0][0],
+                        bars->vote_end, &bars->half_max[0][0][0], &bars->half_ref[0][0][0]};
+    softmax_tile<D, BK>(a, x, y, abort);
   }
 
   tc_fence_before();

@@ -72,19 +72,28 @@ def run(keep, skip, rescale, rng):
         while not q_full.ready(0, 0):
             yield
         kept = 0
-        for u in range(n_comp):
-            while not k_full.ready(u & 1, u):
+        if n_comp:
+            while not k_full.ready(0, 0):
                 yield
-            pending.append(("mma", [s_full, k_empty]))            # S(u); the K slot is free after it
+            pending.append(("mma", [s_full, k_empty]))            # S(0); the K slot is free after it
+        for u in range(n_comp):
             while not p_full[u & 1].ready((u >> 1) & 1, u >> 1):
                 yield
             while not v_full.ready(u & 1, u):
                 yield
+            bars = []
             if not skip[u]:
-                pending.append(("mma", [v_empty, o_done[kept & 1]]))   # P V(u)
+                pending.append(("mma", []))                       # P V(u), committed below
+                bars += [v_empty, o_done[kept & 1]]
                 kept += 1
             else:
                 v_empty.arrive()
+            if u + 1 < n_comp:
+                # S(u + 1) is issued right behind P V(u), before the commits
+                while not k_full.ready((u + 1) & 1, u + 1):
+                    yield
+                bars += [s_full, k_empty]
+            pending.append(("mma", bars))                         # the commits: after every MMA so far
         pending.append(("mma", [drain]))
         while not drain.ready(0, 0):
             yield
