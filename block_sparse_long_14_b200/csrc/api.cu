@@ -80,7 +80,8 @@ const int32_t* cu_kblocks(const cosa_shape_t& s) { return s.kv_lens != nullptr ?
 // [Hkv, NKB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d], and the
 // q-block vectors' max-abs [Hq, NQB] (the Top-p cut's logit scale).
 struct WsLayout {
-  size_t kq_off, ks_off, qa_off, qm_off, total;
+  size_t kq_off, ks_off, qa_off, qm_off, cand_off, hrmj_off, total;
+  int cand_stride;   // candidates per row of the score rows (0: no score rows)
 };
 
 WsLayout ws_layout(const cosa_shape_t& s) {
@@ -92,7 +93,12 @@ WsLayout ws_layout(const cosa_shape_t& s) {
   const size_t qa_bytes =
       static_cast<size_t>(s.num_q_heads) * s.total_qblocks * (s.block_size / 16 + 1) * s.head_dim;
   w.qm_off = align_up(w.qa_off + qa_bytes, 256);
-  w.total = align_up(w.qm_off + static_cast<size_t>(s.num_q_heads) * s.total_qblocks * 4, 256);
+  w.cand_off = align_up(w.qm_off + static_cast<size_t>(s.num_q_heads) * s.total_qblocks * 4, 256);
+  // head_dim 128: every row's candidate score bits [Hq, NQB, NKB_max] and HRM blocks [Hq, NQB, 8]
+  w.cand_stride = s.head_dim == 128 ? ceil_div(s.max_seqlen, s.block_size) : 0;
+  w.hrmj_off = align_up(w.cand_off + static_cast<size_t>(s.num_q_heads) * s.total_qblocks * w.cand_stride * 4, 256);
+  w.total = align_up(w.hrmj_off + (w.cand_stride > 0 ? static_cast<size_t>(s.num_q_heads) * s.total_qblocks * 32 : 0),
+                     256);
   return w;
 }
 
@@ -250,6 +256,36 @@ int proxy_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   sa.qm = reinterpret_cast<float*>(ws + w.qm_off);
   sa.top_p = top_p;
   const int GT = proxy_group(*shape);
+  int q_stages = 0;
+  if (shape->head_dim == 128 && top_p == 0.0f && w.cand_stride > 0 &&
+      stream_fits(GT, shape->block_size / 16, sa.npow2_max, kmax, &q_stages) &&
+      select_rows_smem_bytes(sa.npow2_max, kmax) <= 200 * 1024) {
+    // the budget cut at head_dim 128: pooling, scores and HRM flags in one persistent kernel,
+    // then the selection of every row, one warp each
+    CUtensorMap q_map, kq_map;
+    {
+      // Q as (d, query head, token): a box is 16 rows of a tile's GT heads
+      const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(shape->num_q_heads),
+                                  static_cast<cuuint64_t>(shape->total_tokens)};
+      const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(shape->num_q_heads) * 256};
+      const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(GT), 16};
+      if (!make_map(&q_map, q, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return COSA_ERR_CUDA;
+    }
+    {
+      // int8 key vectors as a [Hkv * NKB, 128] byte matrix, 128 key blocks per score tile
+      const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(shape->num_kv_heads) * total_kblocks(*shape)};
+      const cuuint64_t strides[1] = {128};
+      const cuuint32_t box[2] = {128, 128};
+      if (!make_map(&kq_map, sa.kq, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return COSA_ERR_CUDA;
+    }
+    sa.cand = reinterpret_cast<uint32_t*>(ws + w.cand_off);
+    sa.hrmj = reinterpret_cast<int32_t*>(ws + w.hrmj_off);
+    sa.cand_stride = w.cand_stride;
+    const StreamLayout lay = stream_layout(GT, shape->block_size / 16, sa.npow2_max, kmax, q_stages);
+    if (launch_stream(sa, GT, q_map, kq_map, lay, st) != cudaSuccess) return COSA_ERR_CUDA;
+    return launch_select_rows(sa, st) == cudaSuccess ? COSA_OK : COSA_ERR_CUDA;
+  }
   sa.scratch_bytes = select_scratch_bytes(*shape, kmax, GT, sa.npow2_max);
   if (launch_qpool(sa, GT, st) != cudaSuccess) return COSA_ERR_CUDA;
   if (shape->head_dim == 128) {

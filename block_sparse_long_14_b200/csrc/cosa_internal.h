@@ -45,6 +45,9 @@ struct ScoreArgs {
   int scratch_bytes;   // radix-select scratch of the select kernel
   float* qm;           // [Hq, NQB] max-abs of each q-block sum vector (written by qpool; nullable)
   float top_p;         // 0: budget cut k_i from bp; in (0, 1]: Top-p cut (reads qm)
+  uint32_t* cand;      // [Hq, NQB, cand_stride] score bits of each candidate (persistent proxy path)
+  int32_t* hrmj;       // [Hq, NQB, 8] the HRM blocks of each row, -1 padded (persistent proxy path)
+  int cand_stride;     // candidates per row the cand rows hold (the longest sequence's key blocks)
 };
 
 struct RemapArgs {
@@ -93,6 +96,26 @@ cudaError_t launch_select(const ScoreArgs& a, int GT, cudaStream_t stream);   //
 // a.qa -> lists on tcgen05 int8 MMAs (head_dim 128); kq_map covers a.kq as [Hkv * NQB, 128] int8
 cudaError_t launch_select_tc(const ScoreArgs& a, int GT, const CUtensorMap& kq_map, cudaStream_t stream);
 size_t select_tc_smem_bytes(int GT, int npow2_max, int scratch_bytes);
+// The persistent proxy kernel (head_dim 128, budget cut): pooling, scores and
+// HRM flags of every tile in one launch, one CTA per SM, writing a.cand and
+// a.hrmj.  Shared-memory layout (byte offsets from a 1024-aligned base; ks and
+// red are those of epilogue group 0, group 1's follow group_bytes later) and
+// its limit:
+struct StreamLayout {
+  uint32_t q, k, a, ks, red, group_bytes, bars, total;
+  int q_stages;   // Q chunks in flight (16 rows each)
+};
+constexpr uint32_t kStreamSmemLimit = 227 * 1024;
+StreamLayout stream_layout(int GT, int R, int npow2_max, int kmax, int q_stages);
+// Deepest Q ring that fits (true), or false when even 3 stages do not.
+bool stream_fits(int GT, int R, int npow2_max, int kmax, int* q_stages);
+// q_map: Q as (d, Hq, T) with boxes of (128, GT, 16), no swizzle; kq_map: the
+// pooled keys as [Hkv * NKB, 128] int8 in boxes of 128 rows, 128B swizzle.
+cudaError_t launch_stream(const ScoreArgs& a, int GT, const CUtensorMap& q_map, const CUtensorMap& kq_map,
+                          const StreamLayout& lay, cudaStream_t stream);
+// Selection of every row from a.cand / a.hrmj (one warp per (head, q-block) row): the ordered lists.
+cudaError_t launch_select_rows(const ScoreArgs& a, cudaStream_t stream);
+size_t select_rows_smem_bytes(int npow2_max, int kmax);
 cudaError_t launch_remap(const RemapArgs& a, cudaStream_t stream);
 cudaError_t launch_osk(const OskArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
                        const CUtensorMap& vmap, int head_dim, cudaStream_t stream);

@@ -19,12 +19,20 @@ static constexpr float kTiny = 1.17549435e-38f;  // 2^-126: smallest normal fp32
 // Sort key: bit 63 = not HRM, bits 31..62 = score mapped to an unsigned
 // order that is descending in the score, bits 0..30 = block index.
 // Ascending keys give (HRM first, score descending, index ascending).
-__device__ __forceinline__ uint64_t make_key(float sc, int j) {
+// The score bits of a sort key: an unsigned order descending in the score.
+__device__ __forceinline__ uint32_t score_bits(float sc) {
   uint32_t u = __float_as_uint(sc);
   if ((u & 0x7FFFFFFFu) == 0) u = 0;                         // -0 -> +0
   const uint32_t asc = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return (1ull << 63) | (static_cast<uint64_t>(~asc) << 31) | static_cast<uint32_t>(j);
+  return ~asc;
 }
+
+// The sort key of a non-HRM block j from its score bits.
+__device__ __forceinline__ uint64_t key_of(uint32_t bits, int j) {
+  return (1ull << 63) | (static_cast<uint64_t>(bits) << 31) | static_cast<uint32_t>(j);
+}
+
+__device__ __forceinline__ uint64_t make_key(float sc, int j) { return key_of(score_bits(sc), j); }
 
 // The score a sort key was made from (make_key is a bijection on non-zero
 // floats and maps both zeros to +0).
@@ -223,6 +231,80 @@ static __device__ int warp_select_smallest(const uint64_t* kr, int n, int k_i, i
     }
   }
   return min(cnt, k_i);
+}
+
+// The k smallest of n unique 64-bit keys kr[0..n) by one warp, for k small
+// against n: 64 keys taken at evenly spaced positions are sorted in registers
+// (warp bitonic network); a threshold T is the sample at a rank that puts
+// about 2k keys at or below it; one pass compacts every key <= T into
+// buf (ballot); if fewer than k were kept the rank is raised and the pass
+// repeated (on the 128K layer at a 5% budget: 4% of the rows, and the kept
+// set is 1.9 k at the median).  The kept set, padded with ~0 to a power of two, is sorted in
+// shared memory and its first k keys are exactly the k smallest.  Requires
+// 1 <= k < n.  Returns the number of kept keys (>= k), or -1 when the kept
+// set would exceed `cap` keys or no sample reaches k (the caller then uses
+// warp_select_smallest).
+static __device__ int warp_select_sampled(const uint64_t* kr, int n, int k, uint64_t* buf, int cap) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  // sample element e = 2 lane + s, taken at position (e n) / 64
+  uint64_t v0 = kr[(2 * lane * n) >> 6], v1 = kr[((2 * lane + 1) * n) >> 6];
+  for (int kk = 2; kk <= 64; kk <<= 1) {
+    const bool asc = ((2 * lane) & kk) == 0;      // this lane's elements sit in an ascending run
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      if (j == 1) {
+        if ((v0 > v1) == asc) {
+          const uint64_t t = v0;
+          v0 = v1;
+          v1 = t;
+        }
+      } else {
+        // partner elements e ^ j: the same slot in lane ^ (j / 2)
+        const uint64_t p0 = __shfl_xor_sync(kFull, v0, j >> 1), p1 = __shfl_xor_sync(kFull, v1, j >> 1);
+        const bool keep_min = ((lane & (j >> 1)) == 0) == asc;
+        v0 = keep_min ? (v0 < p0 ? v0 : p0) : (v0 > p0 ? v0 : p0);
+        v1 = keep_min ? (v1 < p1 ? v1 : p1) : (v1 > p1 ? v1 : p1);
+      }
+    }
+  }
+  int r = min(63, (64 * k + n - 1) / n + 1);   // about 2k keys at or below the r-th sample (the sample
+                                                // spacing is n / 64 ranks)
+  int cnt = 0;
+  for (int attempt = 0;; ++attempt) {
+    const uint64_t t0 = __shfl_sync(kFull, v0, r >> 1), t1 = __shfl_sync(kFull, v1, r >> 1);
+    const uint64_t T = (r & 1) ? t1 : t0;
+    cnt = 0;
+    for (int base = 0; base < n; base += 32) {   // every lane takes every iteration
+      const int x = base + lane;
+      const uint64_t key = x < n ? kr[x] : ~0ull;
+      const bool keep = x < n && key <= T;
+      const unsigned bal = __ballot_sync(kFull, keep);
+      const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+      if (keep && pos < cap) buf[pos] = key;
+      cnt += __popc(bal);
+    }
+    if (cnt >= k || r == 63 || attempt == 2) break;
+    r = min(63, r + r / 2 + 2);
+  }
+  if (cnt < k || cnt > cap) return -1;
+  int P = 1;
+  while (P < cnt) P <<= 1;
+  for (int t = cnt + lane; t < P; t += 32) buf[t] = ~0ull;
+  __syncwarp();
+  for (int kk = 2; kk <= P; kk <<= 1) {
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      for (int i = lane; i < (P >> 1); i += 32) {
+        const int x = ((i & ~(j - 1)) << 1) | (i & (j - 1));   // lower element of pair i
+        const uint64_t va = buf[x], vb = buf[x + j];
+        if ((va > vb) == ((x & kk) == 0)) {
+          buf[x] = vb;
+          buf[x + j] = va;
+        }
+      }
+      __syncwarp();
+    }
+  }
+  return cnt;
 }
 
 }  // namespace cosa

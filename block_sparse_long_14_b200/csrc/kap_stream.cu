@@ -1,0 +1,592 @@
+// The Kernel-Aware Proxy as one persistent kernel (head_dim 128, budget cut).
+//
+// "CoSA: Accelerating Long-Context Inference via Proxy-Kernel Co-Designed
+// Sparse Attention", §5.1 (scoring and pooling run as one fused kernel),
+// §4.2 (block ranking, flag-grouped sorting) and Appendix C.1 / Figure A (HRM
+// group first, then the rest, each by score, cut to the stage-1 budget).
+//
+// One CTA per SM walks its share of the tiles (q-block x group of GT query
+// heads sharing a kv head, longest rows first).  The work of a tile moves
+// through warp roles connected by mbarriers, so that consecutive tiles
+// overlap: while the epilogue warps rank and select tile X, the pooling
+// warps already sum the query rows of tile X+1, whose chunks stream in by TMA.
+//   warp 0      Q producer: the tile's rows in chunks of 16 (one sub-row,
+//               GT heads x 128 dims, 4 KiB per head) into a ring of QS slots.
+//   warp 1      key producer: the pooled int8 key blocks of the tile's kv head,
+//               128 blocks (16 KiB, 128B swizzle) per score tile, 3 slots.
+//   warps 2-5   pooling, one query head each: the fp32 sum of each 16-row
+//               sub-row token by token, the q-block sum as their fold, int8
+//               quantisation, written as the MMA's B operand (double-buffered
+//               across tiles).
+//   warp 6      MMA issuer: D[j][v] = Kq_j . q_v (s8 x s8 -> exact s32) with
+//               tcgen05 kind::i8, 128 key blocks in M (one TMEM lane each) and
+//               the tile's GT (R + 1) vectors in N, into one of two TMEM
+//               accumulators.
+//   warps 7-14  epilogue, two groups of four warps (TMEM lane quadrants 3, 0,
+//               1, 2 and 3, 0, 1, 2) taking alternate tiles: each lane turns
+//               one key block's dots into its score bits per head (written to
+//               the workspace row of that head) and updates the sub-rows'
+//               running argmax; the group then reduces the argmax to the HRM
+//               blocks of each head (written next to the scores).
+// The selection runs in its own kernel (select_rows_kernel): one warp per
+// (head, q-block) row, many rows per SM, a sampled threshold and a sort of the
+// few keys below it (a radix select when that does not fit).
+// Scores, flags and lists are bit-identical to the two-stage kernels: the same
+// fp32 operations in the same order, and integer dots.  Every wait is bounded;
+// on expiry the CTA records COSA_ERR_TIMEOUT, lets its own copies and MMAs
+// land, frees TMEM and exits.
+#include <cstdint>
+
+#include "cosa_device.cuh"
+#include "cosa_internal.h"
+#include "kap_common.cuh"
+
+namespace cosa {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kThreads = 480;
+constexpr int kQWarp = 0, kKWarp = 1, kPoolWarp0 = 2, kMmaWarp = 6, kEpiWarp0 = 7;
+constexpr int kEpiThreads = 128;     // one epilogue group
+constexpr int kEpiBar0 = 2;          // named barriers 2 and 3: the two epilogue groups
+constexpr int kSelCap = 256;         // kept keys per row of the sampled selection
+constexpr int kRowWarps = 8;         // rows per CTA of the selection kernel
+constexpr int kKeys = 128;           // key blocks per score tile
+constexpr int kKStages = 3;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+__host__ __device__ constexpr int stream_np(int GT, int R) { return (GT * (R + 1) + 15) / 16 * 16; }
+
+template <int GT, int R>
+struct Shape {
+  static constexpr int NV = GT * (R + 1);          // query vectors of a tile
+  static constexpr int NP = stream_np(GT, R);      // MMA N (a multiple of 16)
+  static constexpr int NS = GT * R;                // sub-rows of a tile
+  static constexpr int ACC = NP <= 32 ? 32 : 64;   // TMEM columns per accumulator
+  static constexpr int TMEM_COLS = 4 * ACC;         // two accumulators per epilogue group
+  static constexpr int QSLOT = 16 * GT * kD * 2;   // one chunk: 16 rows x GT heads x d bf16
+  static constexpr int KSLOT = kKeys * kD;         // one score tile of int8 key vectors
+  static constexpr int ASLOT = NP * kD;            // the int8 query vectors (B operand)
+  static constexpr uint32_t IDESC = idesc_s8_s32(kKeys, NP);
+};
+
+struct Bars {
+  uint64_t q_full[8], q_empty[8];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t a_full[2], a_empty[2];
+  uint64_t acc_full[4], acc_empty[4];   // [2 group + buffer]
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// The pooling warps' int8 vector of one lane (4 dims) into row `row` of the
+// 128B-swizzled B operand.
+__device__ __forceinline__ void store_vec(unsigned char* amat, int row, int lane, uint32_t packed) {
+  *reinterpret_cast<uint32_t*>(amat + row * 128 + (((lane >> 2) ^ (row & 7)) << 4) + (lane & 3) * 4) = packed;
+}
+
+// int8 quantisation of a vector spread over a warp (4 dims per lane): M = max |x|,
+// x -> rint(x * (127 / M)) with both operations rounded to nearest; M below the
+// normal range gives zeros.  Returns the lane's 4 codes packed, and M.
+__device__ __forceinline__ uint32_t quantize4(const float (&x)[4], float& M_out) {
+  float M = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) M = fmaxf(M, fabsf(x[e]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float inv = (M < kTiny) ? 0.0f : __fdiv_rn(127.0f, M);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int q = static_cast<int>(rintf(__fmul_rn(x[e], inv)));
+    packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * e);
+  }
+  M_out = M;
+  return packed;
+}
+
+}  // namespace
+
+template <int GT, int R>
+__global__ void __launch_bounds__(kThreads, 1)
+    kap_stream_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap kq_map,
+                      const ScoreArgs a, const StreamLayout lay) {
+  using S = Shape<GT, R>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) report(a.status, kErrBounds, 0x2F0);
+    return;
+  }
+  unsigned char* sQ = smem + lay.q;
+  unsigned char* sK = smem + lay.k;
+  unsigned char* sA = smem + lay.a;
+  // per epilogue group: key scales [npow2_max], sub-row maxima [4][NS]
+  float* sKs0 = reinterpret_cast<float*>(smem + lay.ks);
+  uint64_t* red0 = reinterpret_cast<uint64_t*>(smem + lay.red);
+  Bars* bars = reinterpret_cast<Bars*>(smem + lay.bars);
+  volatile int* abort = &bars->abort;
+  const int QS = lay.q_stages;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ntiles = a.nqb_total * (a.num_q_heads / GT);
+  const int b = a.block_size;
+
+  if (tid == 0) {
+    for (int x = 0; x < QS; ++x) {
+      mbar_init(&bars->q_full[x], 1);
+      mbar_init(&bars->q_empty[x], 4);            // the four pooling warps
+    }
+    for (int x = 0; x < kKStages; ++x) {
+      mbar_init(&bars->k_full[x], 1);
+      mbar_init(&bars->k_empty[x], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->a_full[x], 4);             // the four pooling warps
+      mbar_init(&bars->a_empty[x], 1);
+    }
+    for (int x = 0; x < 4; ++x) {
+      mbar_init(&bars->acc_full[x], 1);
+      mbar_init(&bars->acc_empty[x], 4);          // the four warps of the group
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    mbar_fence_init();
+  }
+  // the padding rows of both B-operand buffers stay zero
+  for (int x = tid; x < 2 * (S::NP - S::NV) * 32; x += kThreads) {
+    const int buf = x / ((S::NP - S::NV) * 32), rem = x % ((S::NP - S::NV) * 32);
+    reinterpret_cast<uint32_t*>(sA + buf * S::ASLOT + S::NV * 128)[rem] = 0u;
+  }
+  fence_proxy_async();
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars->tmem_base, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == kQWarp) {
+    // ======================================================== Q producer
+    if (lane == 0) {
+      prefetch_tmap(&q_map);
+      int qc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const Tile tl = tile_at<GT>(a, tile);
+        if (tl.bad || tl.npow2 > a.npow2_max) continue;
+        for (int v = 0; v < R && ok; ++v, ++qc) {
+          const int slot = qc % QS, use = qc / QS;
+          if (use >= 1) ok = mbar_wait(&bars->q_empty[slot], (use - 1) & 1, kWaitLimit, abort, a.status, 0x230);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars->q_full[slot], S::QSLOT);
+          // rows outside the tile's present rows (or the tensor) are loaded but never summed
+          tma_load_3d(sQ + slot * S::QSLOT, &q_map, &bars->q_full[slot], 0, tl.h0,
+                      static_cast<int>(tl.q_row0 + static_cast<long>(tl.i) * b + 16 * v));
+        }
+      }
+      // every chunk requested has landed before the CTA exits
+      for (int c = max(0, qc - QS); c < qc; ++c) mbar_drain(&bars->q_full[c % QS], (c / QS) & 1);
+    }
+  } else if (warp == kKWarp) {
+    // ======================================================== key producer
+    if (lane == 0) {
+      prefetch_tmap(&kq_map);
+      int kc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const Tile tl = tile_at<GT>(a, tile);
+        if (tl.bad || tl.npow2 > a.npow2_max) continue;
+        const int ntk = (tl.n + kKeys - 1) / kKeys;
+        const int row0 = tl.kv * a.nkb_total + tl.kb0;
+        for (int kt = 0; kt < ntk && ok; ++kt, ++kc) {
+          const int slot = kc % kKStages, use = kc / kKStages;
+          if (use >= 1) ok = mbar_wait(&bars->k_empty[slot], (use - 1) & 1, kWaitLimit, abort, a.status, 0x231);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars->k_full[slot], S::KSLOT);
+          // key blocks past the row's candidates are loaded but never read
+          tma_load_2d(sK + slot * S::KSLOT, &kq_map, &bars->k_full[slot], 0, row0 + kt * kKeys);
+        }
+      }
+      for (int c = max(0, kc - kKStages); c < kc; ++c) mbar_drain(&bars->k_full[c % kKStages], (c / kKStages) & 1);
+    }
+  } else if (warp < kMmaWarp) {
+    // ======================================================== pooling (one query head per warp)
+    const int pw = warp - kPoolWarp0;
+    int qc = 0, tcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+      const Tile tl = tile_at<GT>(a, tile);
+      if (tl.bad || tl.npow2 > a.npow2_max) continue;
+      const int buf = tcount & 1;
+      if (tcount >= 2)
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->a_empty[buf], ((tcount >> 1) - 1) & 1, kWaitLimit,
+                                                     abort, a.status, 0x232));
+      unsigned char* amat = sA + buf * S::ASLOT;
+      float blk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int v = 0; v < R; ++v, ++qc) {
+        const int slot = qc % QS;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->q_full[slot], (qc / QS) & 1, kWaitLimit, abort,
+                                                     a.status, 0x233));
+        if (ok && pw < GT) {
+          // sub-row v: rows 16v .. 16v + 15 of the tile, summed token by token (present rows
+          // only); all 16 rows are read first so the loads overlap
+          const unsigned char* src = sQ + slot * S::QSLOT + pw * (kD * 2) + lane * 8;
+          uint2 raw[16];
+#pragma unroll
+          for (int rr = 0; rr < 16; ++rr) raw[rr] = *reinterpret_cast<const uint2*>(src + rr * (GT * kD * 2));
+          const int lo_row = tl.rlo - 16 * v, hi_row = tl.rhi - 16 * v;   // present rows [lo_row, hi_row)
+          float sub[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int rr = 0; rr < 16; ++rr) {
+            if (rr >= lo_row && rr < hi_row) {
+              sub[0] = __fadd_rn(sub[0], __uint_as_float(raw[rr].x << 16));
+              sub[1] = __fadd_rn(sub[1], __uint_as_float(raw[rr].x & 0xFFFF0000u));
+              sub[2] = __fadd_rn(sub[2], __uint_as_float(raw[rr].y << 16));
+              sub[3] = __fadd_rn(sub[3], __uint_as_float(raw[rr].y & 0xFFFF0000u));
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) blk[e] = __fadd_rn(blk[e], sub[e]);   // the q-block sum: their fold
+          float M;
+          const uint32_t packed = quantize4(sub, M);
+          store_vec(amat, pw * (R + 1) + 1 + v, lane, packed);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_empty[slot]);
+      }
+      if (ok && pw < GT) {
+        float M;
+        const uint32_t packed = quantize4(blk, M);
+        store_vec(amat, pw * (R + 1), lane, packed);
+        if (a.qm != nullptr && lane == 0) a.qm[static_cast<long>(tl.h0 + pw) * a.nqb_total + tl.I] = M;
+      }
+      fence_proxy_async();   // the generic-proxy stores reach the tensor core's view of shared memory
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->a_full[buf]);
+      ++tcount;
+    }
+  } else if (warp == kMmaWarp) {
+    // ======================================================== MMA issuer
+    if (lane == 0) {
+      int kc = 0, tcount = 0;
+      int accg[2] = {0, 0};   // key tiles issued to each epilogue group
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const Tile tl = tile_at<GT>(a, tile);
+        if (tl.bad || tl.npow2 > a.npow2_max) continue;
+        const int buf = tcount & 1, eg = tcount & 1;   // the tile's B-operand buffer and epilogue group
+        ok = mbar_wait(&bars->a_full[buf], (tcount >> 1) & 1, kWaitLimit, abort, a.status, 0x234);
+        if (!ok) break;
+        const uint32_t a_base = smem_u32(sA + buf * S::ASLOT);
+        const int ntk = (tl.n + kKeys - 1) / kKeys;
+        for (int kt = 0; kt < ntk; ++kt, ++kc) {
+          const int slot = kc % kKStages;
+          const int u = accg[eg], ab = 2 * eg + (u & 1);
+          ok = mbar_wait(&bars->k_full[slot], (kc / kKStages) & 1, kWaitLimit, abort, a.status, 0x235);
+          if (ok && u >= 2)
+            ok = mbar_wait(&bars->acc_empty[ab], ((u >> 1) - 1) & 1, kWaitLimit, abort, a.status, 0x236);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(sK + slot * S::KSLOT);
+#pragma unroll
+          for (int ks = 0; ks < kD / 32; ++ks)
+            tc_mma_i8(tmem + ab * S::ACC, sw128_desc(k_base + ks * 32, 16, 1024), sw128_desc(a_base + ks * 32, 16, 1024),
+                      S::IDESC, ks > 0 ? 1u : 0u);
+          tc_commit(&bars->k_empty[slot]);   // the key slot is free once these MMAs complete
+          tc_commit(&bars->acc_full[ab]);
+          ++accg[eg];
+        }
+        if (!ok) break;
+        tc_commit(&bars->a_empty[buf]);      // the tile's vectors are read
+        ++tcount;
+      }
+      // every MMA issued here completes before TMEM is freed
+      tc_commit(&bars->drain);
+      mbar_drain(&bars->drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ======================================================== epilogue: scores and HRM flags
+    const int eg = (warp - kEpiWarp0) >> 2;      // epilogue group: takes the CTA's tiles of parity eg
+    const int et = tid - (kEpiWarp0 + 4 * eg) * 32;   // 0..127
+    const int ew = (warp - kEpiWarp0) & 3;
+    const int bar = kEpiBar0 + eg;
+    const int quad = warp & 3;                   // TMEM lane quadrant
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+    float* sKs = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(sKs0) + eg * lay.group_bytes);
+    uint64_t* red = red0 + eg * (lay.group_bytes / 8);
+    int u = 0, kloc = 0;   // key tiles consumed by this group; this CTA's good tiles so far
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+      const Tile tl = tile_at<GT>(a, tile);
+      if (tl.bad || tl.npow2 > a.npow2_max) {
+        if (et == 0 && eg == 0) report(a.status, kErrBounds, 0x237);
+        continue;
+      }
+      if ((kloc++ & 1) != eg) continue;
+      const int n = tl.n;
+      const float* ks_row = a.ks + static_cast<long>(tl.kv) * a.nkb_total + tl.kb0;
+      for (int x = et; x < n; x += kEpiThreads) sKs[x] = __ldg(ks_row + x);
+      named_bar_sync(bar, kEpiThreads);
+      uint32_t* cand_row = a.cand + (static_cast<long>(tl.h0) * a.nqb_total + tl.I) * a.cand_stride;
+      const long cand_head = static_cast<long>(a.nqb_total) * a.cand_stride;   // one head further
+
+      uint64_t best[S::NS];
+#pragma unroll
+      for (int x = 0; x < S::NS; ++x) best[x] = 0ull;
+      const int ntk = (n + kKeys - 1) / kKeys;
+      for (int kt = 0; kt < ntk; ++kt, ++u) {
+        const int ab = 2 * eg + (u & 1);
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->acc_full[ab], (u >> 1) & 1, kWaitLimit, abort,
+                                                     a.status, 0x238));
+        if (!ok) continue;
+        tc_fence_after();
+        const int j = kt * kKeys + 32 * quad + lane;         // this lane's key block
+        const float ksj = j < n ? sKs[j] : 0.0f;
+        // this lane's dots, 16 columns at a time: column mt (R + 1) is head mt's block
+        // vector (its score bits), the next R its sub-rows (their running argmax)
+#pragma unroll
+        for (int c = 0; c < S::NP / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(lane_base + ab * S::ACC + c * 16, r);
+          tc_wait_ld();
+          if (c == S::NP / 16 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);   // the accumulator may be overwritten
+          }
+          if (j < n) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int col = c * 16 + e;
+              if (col >= S::NV) continue;
+              const int mt = col / (R + 1), v = col % (R + 1);
+              const float sv = __fmul_rn(static_cast<float>(static_cast<int>(r[e])), ksj);
+              if (v == 0) {
+                cand_row[mt * cand_head + j] = score_bits(sv);
+              } else {
+                const uint64_t cand = pack_best(sv, j);
+                if (cand > best[mt * R + v - 1]) best[mt * R + v - 1] = cand;
+              }
+            }
+          }
+        }
+      }
+      // each sub-row's best over the warp's 32 lanes, then over the group's four warps
+#pragma unroll
+      for (int x = 0; x < S::NS; ++x) {
+        uint64_t v = best[x];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
+          v = o > v ? o : v;
+        }
+        if (lane == 0) red[ew * S::NS + x] = v;
+      }
+      named_bar_sync(bar, kEpiThreads);
+      // the HRM blocks: each present sub-row's argmax (8 slots per head, -1 where none)
+      if (et < GT * 8 && ok) {
+        const int mt = et / 8, sr = et % 8;
+        int jv = -1;
+        if (sr < R) {
+          uint64_t v = red[mt * R + sr];
+#pragma unroll
+          for (int w = 1; w < 4; ++w) v = red[w * S::NS + mt * R + sr] > v ? red[w * S::NS + mt * R + sr] : v;
+          const int jj = static_cast<int>(~static_cast<uint32_t>(v));
+          if (v != 0ull && sub_present(tl, sr) && jj >= 0 && jj < n) jv = jj;
+        }
+        a.hrmj[((static_cast<long>(tl.h0 + mt) * a.nqb_total + tl.I) << 3) + sr] = jv;
+      }
+      named_bar_sync(bar, kEpiThreads);   // key scales and maxima are free for the group's next tile
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, S::TMEM_COLS);
+}
+
+// ============================================================ selection of the rows
+// One warp per (query head, q-block) row, longest rows first: the row's n sort
+// keys rebuilt in shared memory from its score bits (block index in the low
+// bits, the HRM blocks' top bit cleared), then its k_i smallest by a sampled
+// threshold (warp_select_sampled; warp_select_smallest when the kept set does
+// not fit), or all n sorted when k_i = n; written as the ordered list.  Each
+// warp owns its shared memory: keys [npow2_max], kept keys [cap], histogram
+// [256]; no CTA-wide synchronisation.
+__global__ void __launch_bounds__(kRowWarps * 32) select_rows_kernel(const ScoreArgs a, int cap) {
+  extern __shared__ __align__(16) unsigned char smem_rows[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t per_warp = static_cast<size_t>(a.npow2_max + cap) * 8 + 256 * 4;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem_rows + warp * per_warp);
+  uint64_t* sel = keys + a.npow2_max;
+  int* hist = reinterpret_cast<int*>(sel + cap);
+  const long rr = static_cast<long>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  if (rr >= static_cast<long>(a.num_q_heads) * a.nqb_total) return;
+  const int I = a.nqb_total - 1 - static_cast<int>(rr / a.num_q_heads);
+  const int h = static_cast<int>(rr % a.num_q_heads);
+  const int s = find_seq(a.cu_qblocks, a.batch, I);
+  const SeqSpan sp = seq_span(a.cu_seqlens, a.kv_lens, s, a.block_size);
+  const int i = I - __ldg(a.cu_qblocks + s) + sp.i0;
+  const int n = i + 1;
+  if (sp.off < 0 || n > a.npow2_max || n > a.cand_stride) {
+    if (lane == 0) report(a.status, kErrBounds, 0x240);
+    return;
+  }
+  const long row = static_cast<long>(h) * a.nqb_total + I;
+  const uint32_t* cr = a.cand + row * a.cand_stride;
+  for (int x = lane; x < n; x += 32) keys[x] = key_of(__ldg(cr + x), x);
+  __syncwarp();
+  if (lane < 8) {
+    const int j = __ldg(a.hrmj + row * 8 + lane);
+    if (j >= 0 && j < n) atomicAnd(reinterpret_cast<unsigned long long*>(&keys[j]), ~(1ull << 63));
+  }
+  __syncwarp();
+  const int k_i = keep_count(n, a.bp);
+  const uint64_t* out = sel;
+  if (k_i < n) {
+    if (warp_select_sampled(keys, n, k_i, sel, min(cap, kSelCap)) < 0) {
+      int kpow = 1;
+      while (kpow < k_i) kpow <<= 1;
+      if (kpow <= cap) warp_select_smallest(keys, n, k_i, kpow, hist, sel, a.status);
+      else if (lane == 0) report(a.status, kErrBounds, 0x241);   // host sizing forbids it
+    }
+  } else {
+    // every candidate kept: sort them all
+    int P = 1;
+    while (P < n) P <<= 1;
+    for (int t = n + lane; t < P; t += 32) keys[t] = ~0ull;
+    __syncwarp();
+    for (int kk = 2; kk <= P; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        for (int q = lane; q < (P >> 1); q += 32) {
+          const int x = ((q & ~(j - 1)) << 1) | (q & (j - 1));
+          const uint64_t va = keys[x], vb = keys[x + j];
+          if ((va > vb) == ((x & kk) == 0)) {
+            keys[x] = vb;
+            keys[x + j] = va;
+          }
+        }
+        __syncwarp();
+      }
+    }
+    out = keys;
+  }
+  const long o = row * a.kmax;
+  const int k_out = min(k_i, a.kmax);
+  if (k_out < k_i && lane == 0) report(a.status, kErrBounds, 0x242);   // host sizing forbids it
+  for (int t = lane; t < a.kmax; t += 32) {
+    const uint64_t key = t < k_out ? out[t] : 0ull;
+    a.order[o + t] = t < k_out ? static_cast<int32_t>(key & 0x7FFFFFFFu) : -1;
+    a.hrm[o + t] = (t < k_out && !(key >> 63)) ? 1 : 0;
+  }
+  int nh = 0;
+  for (int base = 0; base < k_out; base += 32) {
+    const int t = base + lane;
+    nh += __popc(__ballot_sync(0xffffffffu, t < k_out && !(out[t] >> 63)));
+  }
+  if (lane == 0) {
+    a.count[row] = k_out;
+    a.n_hrm[row] = nh;
+  }
+}
+
+// ============================================================ host side
+StreamLayout stream_layout(int GT, int R, int npow2_max, int kmax, int q_stages) {
+  (void)kmax;
+  const int np = stream_np(GT, R);
+  StreamLayout L{};
+  L.q_stages = q_stages;
+  uint32_t off = 0;
+  L.q = off;
+  off += static_cast<uint32_t>(q_stages) * 16 * GT * kD * 2;
+  L.k = off;
+  off += kKStages * kKeys * kD;
+  L.a = off;
+  off += 2 * np * kD;
+  // one region per epilogue group: key scales, sub-row maxima
+  uint32_t g = 0;
+  L.ks = off + g;
+  g += (static_cast<uint32_t>(npow2_max) * 4 + 15) / 16 * 16;
+  L.red = off + g;
+  g += 4 * GT * R * 8;
+  L.group_bytes = (g + 15) / 16 * 16;
+  off += 2 * L.group_bytes;
+  L.bars = off;
+  off += (sizeof(Bars) + 15) / 16 * 16;
+  L.total = off;
+  return L;
+}
+
+bool stream_fits(int GT, int R, int npow2_max, int kmax, int* q_stages) {
+  for (int qs = 6; qs >= 3; --qs) {
+    if (stream_layout(GT, R, npow2_max, kmax, qs).total <= kStreamSmemLimit) {
+      *q_stages = qs;
+      return true;
+    }
+  }
+  return false;
+}
+
+template <int GT, int R>
+static cudaError_t launch_stream_t(const ScoreArgs& a, const CUtensorMap& q_map, const CUtensorMap& kq_map,
+                                   const StreamLayout& lay, int grid, cudaStream_t stream) {
+  auto kern = kap_stream_kernel<GT, R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(lay.total));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, lay.total, stream>>>(q_map, kq_map, a, lay);
+  return cudaGetLastError();
+}
+
+static int rows_cap(int npow2_max, int kmax) {
+  int kpow = 1;
+  while (kpow < kmax) kpow <<= 1;
+  if (kpow > npow2_max) kpow = npow2_max;
+  return kpow > kSelCap ? kpow : kSelCap;
+}
+
+size_t select_rows_smem_bytes(int npow2_max, int kmax) {
+  return static_cast<size_t>(npow2_max + rows_cap(npow2_max, kmax)) * 8 + 256 * 4;   // one warp's share
+}
+
+cudaError_t launch_select_rows(const ScoreArgs& a, cudaStream_t stream) {
+  const int cap = rows_cap(a.npow2_max, a.kmax);
+  const size_t per_warp = select_rows_smem_bytes(a.npow2_max, a.kmax);
+  int warps = kRowWarps;
+  while (warps > 1 && per_warp * warps > 200 * 1024) warps >>= 1;
+  if (per_warp * warps > 227 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(per_warp * warps));
+  if (e != cudaSuccess) return e;
+  const long rows = static_cast<long>(a.num_q_heads) * a.nqb_total;
+  const unsigned grid = static_cast<unsigned>((rows + warps - 1) / warps);
+  select_rows_kernel<<<grid, warps * 32, per_warp * warps, stream>>>(a, cap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stream(const ScoreArgs& a, int GT, const CUtensorMap& q_map, const CUtensorMap& kq_map,
+                          const StreamLayout& lay, cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int ntiles = a.nqb_total * (a.num_q_heads / GT);
+  const int grid = ntiles < sms ? ntiles : sms;
+  if (grid < 1) return cudaSuccess;
+  const bool b128 = a.block_size == 128;
+  switch (GT) {
+    case 1: return b128 ? launch_stream_t<1, 8>(a, q_map, kq_map, lay, grid, stream)
+                        : launch_stream_t<1, 4>(a, q_map, kq_map, lay, grid, stream);
+    case 2: return b128 ? launch_stream_t<2, 8>(a, q_map, kq_map, lay, grid, stream)
+                        : launch_stream_t<2, 4>(a, q_map, kq_map, lay, grid, stream);
+    default: return b128 ? launch_stream_t<4, 8>(a, q_map, kq_map, lay, grid, stream)
+                         : launch_stream_t<4, 4>(a, q_map, kq_map, lay, grid, stream);
+  }
+}
+
+}  // namespace cosa
