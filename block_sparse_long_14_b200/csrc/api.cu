@@ -77,10 +77,12 @@ int total_kblocks(const cosa_shape_t& s) { return s.kv_lens != nullptr ? s.total
 const int32_t* cu_kblocks(const cosa_shape_t& s) { return s.kv_lens != nullptr ? s.cu_kblocks : s.cu_qblocks; }
 
 // Workspace: status block, pooled int8 keys [Hkv, NKB, d], key scales
-// [Hkv, NKB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d], and the
-// q-block vectors' max-abs [Hq, NQB] (the Top-p cut's logit scale).
+// [Hkv, NKB], pooled int8 query vectors [Hq, NQB, b/16 + 1, d], the q-block
+// vectors' max-abs [Hq, NQB] (the Top-p cut's logit scale) and, at head_dim
+// 128, the score rows, HRM blocks and selection retry list of the
+// persistent proxy.
 struct WsLayout {
-  size_t kq_off, ks_off, qa_off, qm_off, cand_off, hrmj_off, total;
+  size_t kq_off, ks_off, qa_off, qm_off, cand_off, hrmj_off, retry_off, total;
   int cand_stride;   // candidates per row of the score rows (0: no score rows)
 };
 
@@ -97,7 +99,10 @@ WsLayout ws_layout(const cosa_shape_t& s) {
   // head_dim 128: every row's candidate score bits [Hq, NQB, NKB_max] and HRM blocks [Hq, NQB, 8]
   w.cand_stride = s.head_dim == 128 ? ceil_div(s.max_seqlen, s.block_size) : 0;
   w.hrmj_off = align_up(w.cand_off + static_cast<size_t>(s.num_q_heads) * s.total_qblocks * w.cand_stride * 4, 256);
-  w.total = align_up(w.hrmj_off + (w.cand_stride > 0 ? static_cast<size_t>(s.num_q_heads) * s.total_qblocks * 32 : 0),
+  w.retry_off = align_up(w.hrmj_off + (w.cand_stride > 0 ? static_cast<size_t>(s.num_q_heads) * s.total_qblocks * 32 : 0),
+                         256);
+  // the selection's retry list: a count, then up to one entry per row
+  w.total = align_up(w.retry_off + (w.cand_stride > 0 ? 4 * (1 + static_cast<size_t>(s.num_q_heads) * s.total_qblocks) : 0),
                      256);
   return w;
 }
@@ -282,6 +287,7 @@ int proxy_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, co
     sa.cand = reinterpret_cast<uint32_t*>(ws + w.cand_off);
     sa.hrmj = reinterpret_cast<int32_t*>(ws + w.hrmj_off);
     sa.cand_stride = w.cand_stride;
+    sa.retry = reinterpret_cast<int32_t*>(ws + w.retry_off);
     const StreamLayout lay = stream_layout(GT, shape->block_size / 16, sa.npow2_max, kmax, q_stages);
     if (launch_stream(sa, GT, q_map, kq_map, lay, st) != cudaSuccess) return COSA_ERR_CUDA;
     return launch_select_rows(sa, st) == cudaSuccess ? COSA_OK : COSA_ERR_CUDA;

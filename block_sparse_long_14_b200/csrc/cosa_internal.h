@@ -48,6 +48,8 @@ struct ScoreArgs {
   uint32_t* cand;      // [Hq, NQB, cand_stride] score bits of each candidate (persistent proxy path)
   int32_t* hrmj;       // [Hq, NQB, 8] the HRM blocks of each row, -1 padded (persistent proxy path)
   int cand_stride;     // candidates per row the cand rows hold (the longest sequence's key blocks)
+  int32_t* retry;      // [1 + Hq * NQB] rows the register selection leaves to select_rows_kernel
+                       // (retry[0] = how many; nullable: every row by select_rows_kernel)
 };
 
 struct RemapArgs {

@@ -233,45 +233,65 @@ static __device__ int warp_select_smallest(const uint64_t* kr, int n, int k_i, i
   return min(cnt, k_i);
 }
 
+// Ascending bitonic sort of 32 V keys held V per lane by a warp (element e of
+// the sequence is v[e % V] of lane e / V): the in-lane stages compare
+// registers, the others exchange with lane ^ (j / V) by shuffles.
+template <int V>
+__device__ __forceinline__ void warp_sort_regs(uint64_t (&v)[V]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int kk = 2; kk <= 32 * V; kk <<= 1) {
+#pragma unroll
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      if (j < V) {
+#pragma unroll
+        for (int q = 0; q < V; ++q) {
+          const int q2 = q ^ j;
+          if (q2 > q) {
+            const bool asc = ((V * lane + q) & kk) == 0;
+            if ((v[q] > v[q2]) == asc) {
+              const uint64_t t = v[q];
+              v[q] = v[q2];
+              v[q2] = t;
+            }
+          }
+        }
+      } else {
+        const int pl = j / V;
+        const bool keep_min = ((lane & pl) == 0) == (((V * lane) & kk) == 0);
+#pragma unroll
+        for (int q = 0; q < V; ++q) {
+          const uint64_t p = __shfl_xor_sync(0xffffffffu, v[q], pl);
+          v[q] = keep_min ? (v[q] < p ? v[q] : p) : (v[q] > p ? v[q] : p);
+        }
+      }
+    }
+  }
+}
+
 // The k smallest of n unique 64-bit keys kr[0..n) by one warp, for k small
-// against n: 64 keys taken at evenly spaced positions are sorted in registers
-// (warp bitonic network); a threshold T is the sample at a rank that puts
-// about 2k keys at or below it; one pass compacts every key <= T into
-// buf (ballot); if fewer than k were kept the rank is raised and the pass
-// repeated (on the 128K layer at a 5% budget: 4% of the rows, and the kept
-// set is 1.9 k at the median).  The kept set, padded with ~0 to a power of two, is sorted in
-// shared memory and its first k keys are exactly the k smallest.  Requires
-// 1 <= k < n.  Returns the number of kept keys (>= k), or -1 when the kept
-// set would exceed `cap` keys or no sample reaches k (the caller then uses
+// against n: 64 keys taken at evenly spaced positions are sorted in registers;
+// a threshold T is the sample at a rank that puts about 2k keys at or below
+// it; one pass compacts every key <= T into buf (ballot); if fewer than k
+// were kept the rank is raised and the pass repeated (on the 128K layer at a
+// 5% budget: 4% of the rows, and the kept set is 1.9 k at the median).  The
+// kept set, padded with ~0, is sorted (in registers up to 128 keys, else in
+// shared memory as a bitonic network over a power of two) and left in
+// buf[0, cnt): its first k keys are exactly the k smallest.  Requires
+// 1 <= k < n.  Returns the number of kept keys (>= k), or -1 when the kept set
+// would exceed `cap` keys or no sample reaches k (the caller then uses
 // warp_select_smallest).
 static __device__ int warp_select_sampled(const uint64_t* kr, int n, int k, uint64_t* buf, int cap) {
   constexpr unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
-  // sample element e = 2 lane + s, taken at position (e n) / 64
-  uint64_t v0 = kr[(2 * lane * n) >> 6], v1 = kr[((2 * lane + 1) * n) >> 6];
-  for (int kk = 2; kk <= 64; kk <<= 1) {
-    const bool asc = ((2 * lane) & kk) == 0;      // this lane's elements sit in an ascending run
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      if (j == 1) {
-        if ((v0 > v1) == asc) {
-          const uint64_t t = v0;
-          v0 = v1;
-          v1 = t;
-        }
-      } else {
-        // partner elements e ^ j: the same slot in lane ^ (j / 2)
-        const uint64_t p0 = __shfl_xor_sync(kFull, v0, j >> 1), p1 = __shfl_xor_sync(kFull, v1, j >> 1);
-        const bool keep_min = ((lane & (j >> 1)) == 0) == asc;
-        v0 = keep_min ? (v0 < p0 ? v0 : p0) : (v0 > p0 ? v0 : p0);
-        v1 = keep_min ? (v1 < p1 ? v1 : p1) : (v1 > p1 ? v1 : p1);
-      }
-    }
-  }
+  // sample element e = 2 lane + q, taken at position (e n) / 64
+  uint64_t smp[2] = {kr[(2 * lane * n) >> 6], kr[((2 * lane + 1) * n) >> 6]};
+  warp_sort_regs<2>(smp);
   int r = min(63, (64 * k + n - 1) / n + 1);   // about 2k keys at or below the r-th sample (the sample
                                                 // spacing is n / 64 ranks)
   int cnt = 0;
   for (int attempt = 0;; ++attempt) {
-    const uint64_t t0 = __shfl_sync(kFull, v0, r >> 1), t1 = __shfl_sync(kFull, v1, r >> 1);
+    const uint64_t t0 = __shfl_sync(kFull, smp[0], r >> 1), t1 = __shfl_sync(kFull, smp[1], r >> 1);
     const uint64_t T = (r & 1) ? t1 : t0;
     cnt = 0;
     for (int base = 0; base < n; base += 32) {   // every lane takes every iteration
@@ -287,6 +307,19 @@ static __device__ int warp_select_sampled(const uint64_t* kr, int n, int k, uint
     r = min(63, r + r / 2 + 2);
   }
   if (cnt < k || cnt > cap) return -1;
+  __syncwarp();
+  if (cnt <= 128) {
+    uint64_t v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = 4 * lane + q < cnt ? buf[4 * lane + q] : ~0ull;
+    warp_sort_regs<4>(v);
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (4 * lane + q < cnt) buf[4 * lane + q] = v[q];
+    __syncwarp();
+    return cnt;
+  }
   int P = 1;
   while (P < cnt) P <<= 1;
   for (int t = cnt + lane; t < P; t += 32) buf[t] = ~0ull;

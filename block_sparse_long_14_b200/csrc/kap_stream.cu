@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = a.block_size;
 
   if (tid == 0) {
+    if (a.retry != nullptr && blockIdx.x == 0) a.retry[0] = 0;   // the selection's retry list starts empty
     for (int x = 0; x < QS; ++x) {
       mbar_init(&bars->q_full[x], 1);
       mbar_init(&bars->q_empty[x], 4);            // the four pooling warps
@@ -419,15 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // not fit), or all n sorted when k_i = n; written as the ordered list.  Each
 // warp owns its shared memory: keys [npow2_max], kept keys [cap], histogram
 // [256]; no CTA-wide synchronisation.
-__global__ void __launch_bounds__(kRowWarps * 32) select_rows_kernel(const ScoreArgs a, int cap) {
-  extern __shared__ __align__(16) unsigned char smem_rows[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t per_warp = static_cast<size_t>(a.npow2_max + cap) * 8 + 256 * 4;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem_rows + warp * per_warp);
-  uint64_t* sel = keys + a.npow2_max;
-  int* hist = reinterpret_cast<int*>(sel + cap);
-  const long rr = static_cast<long>(blockIdx.x) * (blockDim.x >> 5) + warp;
-  if (rr >= static_cast<long>(a.num_q_heads) * a.nqb_total) return;
+static __device__ void select_row(const ScoreArgs& a, int cap, long rr, uint64_t* keys, uint64_t* sel, int* hist) {
+  const int lane = threadIdx.x & 31;
   const int I = a.nqb_total - 1 - static_cast<int>(rr / a.num_q_heads);
   const int h = static_cast<int>(rr % a.num_q_heads);
   const int s = find_seq(a.cu_qblocks, a.batch, I);
@@ -494,6 +488,168 @@ __global__ void __launch_bounds__(kRowWarps * 32) select_rows_kernel(const Score
     a.count[row] = k_out;
     a.n_hrm[row] = nh;
   }
+}
+
+// Rows r = 0 .. rows - 1 (list == nullptr), else the rows list[1 .. list[0]].
+__global__ void __launch_bounds__(kRowWarps * 32) select_rows_kernel(const ScoreArgs a, int cap, const int32_t* list) {
+  extern __shared__ __align__(16) unsigned char smem_rows[];
+  const int warp = threadIdx.x >> 5;
+  const size_t per_warp = static_cast<size_t>(a.npow2_max + cap) * 8 + 256 * 4;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem_rows + warp * per_warp);
+  uint64_t* sel = keys + a.npow2_max;
+  int* hist = reinterpret_cast<int*>(sel + cap);
+  const long rows = static_cast<long>(a.num_q_heads) * a.nqb_total;
+  const long first = static_cast<long>(blockIdx.x) * (blockDim.x >> 5) + warp;
+  const long stride = static_cast<long>(gridDim.x) * (blockDim.x >> 5);
+  if (list == nullptr) {
+    for (long t = first; t < rows; t += stride) select_row(a, cap, t, keys, sel, hist);
+  } else {
+    const long cnt = min(static_cast<long>(__ldg(list)), rows);
+    for (long t = first; t < cnt; t += stride) {
+      const long rr = __ldg(list + 1 + t);
+      if (rr >= 0 && rr < rows) select_row(a, cap, rr, keys, sel, hist);
+      else if ((threadIdx.x & 31) == 0) report(a.status, kErrBounds, 0x243);
+    }
+  }
+}
+
+// ============================================================ register selection of the rows
+// One warp per row, longest rows first, with no per-row shared-memory copy of
+// the keys: each key is rebuilt from the row's score bits (read from L2, where
+// the score kernel left them) and the row's HRM blocks (held in every lane).
+// Rows of at most 128 candidates are sorted whole in registers; longer rows
+// take a sampled threshold (64 keys at evenly spaced positions, sorted in
+// registers), one ballot pass that compacts the keys at or below it into a
+// 256-key buffer, and a register sort of the kept set.  A row whose kept set
+// does not fit, or whose samples never reach k_i, goes to the retry list
+// (list[0] = length, list[1..] = rows) that select_rows_kernel finishes.
+constexpr int kFastWarps = 8;
+constexpr int kFastCap = 256;
+
+struct RowKeys {
+  const uint32_t* cr;
+  int hb[8];   // the row's HRM blocks (-1: none)
+  __device__ __forceinline__ uint64_t at(int x) const {
+    const uint64_t key = key_of(__ldg(cr + x), x);
+    bool f = false;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) f |= hb[q] == x;
+    return f ? key & ~(1ull << 63) : key;
+  }
+};
+
+// The sorted keys v (element e = V lane + q) as the row's ordered list: the
+// first k_out keys' blocks and HRM flags, -1 / 0 padding up to kmax.
+template <int V>
+__device__ __forceinline__ void emit_row(const ScoreArgs& a, long row, const uint64_t (&v)[V], int k_out) {
+  const int lane = threadIdx.x & 31;
+  const long o = row * a.kmax;
+  int nh = 0;
+#pragma unroll
+  for (int q = 0; q < V; ++q) {
+    const int e = V * lane + q;
+    const bool in = e < k_out;
+    if (e < a.kmax) {
+      a.order[o + e] = in ? static_cast<int32_t>(v[q] & 0x7FFFFFFFu) : -1;
+      a.hrm[o + e] = (in && !(v[q] >> 63)) ? 1 : 0;
+    }
+    nh += __popc(__ballot_sync(0xffffffffu, in && !(v[q] >> 63)));
+  }
+  for (int t = 32 * V + lane; t < a.kmax; t += 32) {
+    a.order[o + t] = -1;
+    a.hrm[o + t] = 0;
+  }
+  if (lane == 0) {
+    a.count[row] = k_out;
+    a.n_hrm[row] = nh;
+  }
+}
+
+// Sort cnt <= 32 V keys (from buf, or from the row itself when buf is null)
+// in registers and emit the first k_out.
+template <int V>
+__device__ __forceinline__ void sort_emit(const ScoreArgs& a, long row, const RowKeys& rk, const uint64_t* buf, int cnt,
+                                          int k_out) {
+  const int lane = threadIdx.x & 31;
+  uint64_t v[V];
+#pragma unroll
+  for (int q = 0; q < V; ++q) {
+    const int e = V * lane + q;
+    v[q] = e < cnt ? (buf != nullptr ? buf[e] : rk.at(e)) : ~0ull;
+  }
+  warp_sort_regs<V>(v);
+  emit_row<V>(a, row, v, k_out);
+}
+
+__global__ void __launch_bounds__(kFastWarps * 32) select_fast_kernel(const ScoreArgs a) {
+  constexpr unsigned kFull = 0xffffffffu;
+  __shared__ uint64_t kept_all[kFastWarps][kFastCap];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* buf = kept_all[warp];
+  const long rr = static_cast<long>(blockIdx.x) * kFastWarps + warp;
+  if (rr >= static_cast<long>(a.num_q_heads) * a.nqb_total) return;
+  const int I = a.nqb_total - 1 - static_cast<int>(rr / a.num_q_heads);
+  const int h = static_cast<int>(rr % a.num_q_heads);
+  const int s = find_seq(a.cu_qblocks, a.batch, I);
+  const SeqSpan sp = seq_span(a.cu_seqlens, a.kv_lens, s, a.block_size);
+  const int n = I - __ldg(a.cu_qblocks + s) + sp.i0 + 1;
+  if (sp.off < 0 || n > a.cand_stride) {
+    if (lane == 0) report(a.status, kErrBounds, 0x244);
+    return;
+  }
+  const long row = static_cast<long>(h) * a.nqb_total + I;
+  RowKeys rk;
+  rk.cr = a.cand + row * a.cand_stride;
+  const int hj = lane < 8 ? __ldg(a.hrmj + row * 8 + lane) : -1;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) rk.hb[q] = __shfl_sync(kFull, hj, q);
+  const int k_i = keep_count(n, a.bp);
+  const int k_out = min(k_i, a.kmax);
+  if (k_out < k_i && lane == 0) report(a.status, kErrBounds, 0x245);   // host sizing forbids it
+
+  if (n <= 64) {
+    sort_emit<2>(a, row, rk, nullptr, n, k_out);
+    return;
+  }
+  if (n <= 128) {
+    sort_emit<4>(a, row, rk, nullptr, n, k_out);
+    return;
+  }
+  int cnt = -1;
+  if (k_i < n) {
+    // sample element e = 2 lane + q, taken at position (e n) / 64
+    uint64_t smp[2] = {rk.at((2 * lane * n) >> 6), rk.at(((2 * lane + 1) * n) >> 6)};
+    warp_sort_regs<2>(smp);
+    int r = min(63, (64 * k_i + n - 1) / n + 1);   // about 2 k_i keys at or below the r-th sample
+    for (int attempt = 0; attempt < 3; ++attempt) {
+      const uint64_t t0 = __shfl_sync(kFull, smp[0], r >> 1), t1 = __shfl_sync(kFull, smp[1], r >> 1);
+      const uint64_t T = (r & 1) ? t1 : t0;
+      cnt = 0;
+      for (int base = 0; base < n; base += 128) {   // four loads in flight per lane
+        uint64_t key[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int x = base + 32 * u + lane;
+          key[u] = x < n ? rk.at(x) : ~0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool keep = base + 32 * u + lane < n && key[u] <= T;
+          const unsigned bal = __ballot_sync(kFull, keep);
+          const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+          if (keep && pos < kFastCap) buf[pos] = key[u];
+          cnt += __popc(bal);
+        }
+      }
+      if (cnt >= k_i || r == 63) break;
+      r = min(63, r + r / 2 + 2);
+    }
+    __syncwarp();
+  }
+  if (cnt >= k_i && cnt <= 64) sort_emit<2>(a, row, rk, buf, cnt, k_out);
+  else if (cnt >= k_i && cnt <= 128) sort_emit<4>(a, row, rk, buf, cnt, k_out);
+  else if (cnt >= k_i && cnt <= kFastCap) sort_emit<8>(a, row, rk, buf, cnt, k_out);
+  else if (lane == 0) a.retry[1 + atomicAdd(a.retry, 1)] = static_cast<int32_t>(rr);
 }
 
 // ============================================================ host side
@@ -564,8 +720,20 @@ cudaError_t launch_select_rows(const ScoreArgs& a, cudaStream_t stream) {
                                        static_cast<int>(per_warp * warps));
   if (e != cudaSuccess) return e;
   const long rows = static_cast<long>(a.num_q_heads) * a.nqb_total;
-  const unsigned grid = static_cast<unsigned>((rows + warps - 1) / warps);
-  select_rows_kernel<<<grid, warps * 32, per_warp * warps, stream>>>(a, cap);
+  long grid = (rows + warps - 1) / warps;
+  if (a.retry != nullptr && a.kmax <= 128) {
+    // the register selection (kept sets of about 2 k_i fit its 256-key buffer), then the
+    // rows it leaves, on a grid of two CTAs per SM
+    select_fast_kernel<<<static_cast<unsigned>((rows + kFastWarps - 1) / kFastWarps), kFastWarps * 32, 0, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    grid = grid < 2L * sms ? grid : 2L * sms;
+    select_rows_kernel<<<static_cast<unsigned>(grid), warps * 32, per_warp * warps, stream>>>(a, cap, a.retry);
+  } else {
+    select_rows_kernel<<<static_cast<unsigned>(grid), warps * 32, per_warp * warps, stream>>>(a, cap, nullptr);
+  }
   return cudaGetLastError();
 }
 

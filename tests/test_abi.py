@@ -148,9 +148,9 @@ def test_cached_prefix_shape_checks(lib):
     assert kmax == kap.kmax_for(1024, 0.05)          # lists sized by the longest key sequence
     n_full, _ = _ws(_shape(), 0.05)
     # pooled keys and scales sized by NKB (same as full prefill); query vectors and their
-    # scales, each row's candidate score bits (the longest sequence's 1024 key blocks) and
-    # its 8 HRM slots by NQB only
-    per_qblock = 32 * 9 * 128 + 32 * 4 + 32 * 1024 * 4 + 32 * 8 * 4
+    # scales, each row's candidate score bits (the longest sequence's 1024 key blocks), its 8
+    # HRM slots and its retry-list entry by NQB only
+    per_qblock = 32 * 9 * 128 + 32 * 4 + 32 * 1024 * 4 + 32 * 8 * 4 + 32 * 4
     assert n_full - n_prefix == (1024 - 64) * per_qblock
     for bad in (dict(cu_kblocks=0), dict(total_kblocks=0), dict(total_kblocks=1023), dict(total_kblocks=63,
                 max_seqlen=8000)):

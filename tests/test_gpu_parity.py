@@ -367,3 +367,50 @@ def test_zero_blocks_and_single_entry_lists(budget, tau):
     o = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, ref["order"],
                 ref["count"], tau)
     print(budget, tau, gu.compare_attn(res, o, w, tau, gu.all_units(w)))
+
+
+def _sample_defeating_workload():
+    """One 64K-token sequence (b = 128: rows of up to 512 candidates), two kv
+    heads, one query head each, with every query token equal.  Each key block
+    is a constant vector s_j u, so block j's proxy score is proportional to
+    s_j.  For the last q-block (n = 512) the 64 threshold samples of the
+    register selection sit at blocks 8e.  Kv head 0 gives those 64 blocks the
+    highest scores: at a 5 % budget (k = 26) no sample rank tried (the 6th,
+    10th and 16th smallest) has k keys at or below it.  Kv head 1 gives them
+    the lowest scores: every sample has more than the 256 keys the kept buffer
+    holds below it.  Both rows must finish in the shared-memory selection."""
+    from synth import from_arrays
+    rng = np.random.default_rng(41)
+    nb, b, d = 512, 128, 128
+    L = nb * b
+    u = np.ones(d, dtype=np.float32) / np.sqrt(d)
+    on = np.zeros(nb, dtype=bool)
+    on[::8] = True
+    hi = 2.0 + 0.5 * rng.random(nb)
+    lo = -1.0 - 0.5 * rng.random(nb)
+    s = np.stack([np.where(on, hi, lo), np.where(on, -hi, -lo)], axis=1)   # [nb, kv head]
+    k = np.repeat(s, b, axis=0)[:, :, None] * u[None, None, :]
+    q = np.broadcast_to(u, (L, 2, d)).astype(np.float32)
+    v = rng.standard_normal((L, 2, d)).astype(np.float32)
+    return from_arrays([q], [k.astype(np.float32)], [v], b, 128, shuffle=True, seed=41)
+
+
+def test_selection_rows_the_register_path_leaves():
+    """Rows whose sampled threshold fails (too few keys below every sample
+    tried, or more than the kept buffer holds) are finished by the
+    shared-memory selection through the retry list: the lists are bit-exact
+    and both constructed rows are on the list."""
+    w = _sample_defeating_workload()
+    d = gu.upload(w)
+    got, kmax, ws = gu.run_proxy(d, 0.05)
+    ref = kap.kap_proxy(w.q, w.k_pages, w.page_table, w.seqlens, w.num_kv_heads, w.block_size, 0.05)
+    assert kmax == ref["kmax"] == 26
+    gu.assert_proxy_equal(got, ref)
+    # the retry list is the workspace's last region: a count, then one entry per row
+    rows = w.num_q_heads * d["batch"].total_qblocks
+    region = (4 * (1 + rows) + 255) // 256 * 256
+    lst = ws[ws.numel() - region:].view(torch.int32).cpu().numpy()
+    listed = set(lst[1:1 + lst[0]].tolist())
+    # rows are numbered (q-blocks from the last) * heads + head: the last q-block's are 0 and 1
+    assert {0, 1} <= listed, (lst[0], sorted(listed)[:8])
+    assert all(0 <= r < rows for r in listed)
