@@ -262,7 +262,9 @@ int proxy_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, co
   sa.top_p = top_p;
   const int GT = proxy_group(*shape);
   int q_stages = 0;
-  if (shape->head_dim == 128 && top_p == 0.0f && w.cand_stride > 0 &&
+  // (the persistent kernel records each sub-row's best score tile in 8 bits: at most 256 score
+  // tiles of 128 key blocks per row)
+  if (shape->head_dim == 128 && top_p == 0.0f && w.cand_stride > 0 && sa.npow2_max <= 256 * 128 &&
       stream_fits(GT, shape->block_size / 16, sa.npow2_max, kmax, &q_stages) &&
       select_rows_smem_bytes(sa.npow2_max, kmax) <= 200 * 1024) {
     // the budget cut at head_dim 128: pooling, scores and HRM flags in one persistent kernel,

@@ -100,16 +100,16 @@ cudaError_t launch_select_tc(const ScoreArgs& a, int GT, const CUtensorMap& kq_m
 size_t select_tc_smem_bytes(int GT, int npow2_max, int scratch_bytes);
 // The persistent proxy kernel (head_dim 128, budget cut): pooling, scores and
 // HRM flags of every tile in one launch, one CTA per SM, writing a.cand and
-// a.hrmj.  Shared-memory layout (byte offsets from a 1024-aligned base; ks and
-// red are those of epilogue group 0, group 1's follow group_bytes later) and
-// its limit:
+// a.hrmj.  Shared-memory layout (byte offsets from a 1024-aligned base: Q
+// ring, key tiles, int8 query vectors, odd sub-row sums; ks and red are those
+// of epilogue group 0, group 1's follow group_bytes later) and its limit:
 struct StreamLayout {
-  uint32_t q, k, a, ks, red, group_bytes, bars, total;
+  uint32_t q, k, a, sub, ks, red, group_bytes, bars, total;
   int q_stages;   // Q chunks in flight (16 rows each)
 };
 constexpr uint32_t kStreamSmemLimit = 227 * 1024;
 StreamLayout stream_layout(int GT, int R, int npow2_max, int kmax, int q_stages);
-// Deepest Q ring that fits (true), or false when even 3 stages do not.
+// Deepest even Q ring (8, 6 or 4 stages) that fits (true), or false when 4 stages do not.
 bool stream_fits(int GT, int R, int npow2_max, int kmax, int* q_stages);
 // q_map: Q as (d, Hq, T) with boxes of (128, GT, 16), no swizzle; kq_map: the
 // pooled keys as [Hkv * NKB, 128] int8 in boxes of 128 rows, 128B swizzle.

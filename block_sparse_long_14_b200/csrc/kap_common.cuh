@@ -90,6 +90,13 @@ __device__ __forceinline__ Tile tile_at(const ScoreArgs& a, int tile) {
   return t;
 }
 
+// x with bits [pos, pos + 8) replaced by the low 8 bits of v.
+__device__ __forceinline__ uint32_t bfi8(uint32_t v, uint32_t x, int pos) {
+  uint32_t d;
+  asm("bfi.b32 %0, %1, %2, %3, 8;" : "=r"(d) : "r"(v), "r"(x), "r"(pos));
+  return d;
+}
+
 // Stage-1 count of a row with n causal candidates: k_i = max(1, ceil(n bp / 10^4)).
 __device__ __forceinline__ int keep_count(int n, int bp) {
   return static_cast<int>(max(1LL, (static_cast<long long>(n) * bp + 9999) / 10000));
@@ -233,11 +240,12 @@ static __device__ int warp_select_smallest(const uint64_t* kr, int n, int k_i, i
   return min(cnt, k_i);
 }
 
-// Ascending bitonic sort of 32 V keys held V per lane by a warp (element e of
-// the sequence is v[e % V] of lane e / V): the in-lane stages compare
-// registers, the others exchange with lane ^ (j / V) by shuffles.
-template <int V>
-__device__ __forceinline__ void warp_sort_regs(uint64_t (&v)[V]) {
+// Ascending bitonic sort of 32 V keys (32- or 64-bit) held V per lane by a
+// warp (element e of the sequence is v[e % V] of lane e / V): the in-lane
+// stages compare registers, the others exchange with lane ^ (j / V) by
+// shuffles.
+template <int V, typename T>
+__device__ __forceinline__ void warp_sort_regs(T (&v)[V]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int kk = 2; kk <= 32 * V; kk <<= 1) {
@@ -250,7 +258,7 @@ __device__ __forceinline__ void warp_sort_regs(uint64_t (&v)[V]) {
           if (q2 > q) {
             const bool asc = ((V * lane + q) & kk) == 0;
             if ((v[q] > v[q2]) == asc) {
-              const uint64_t t = v[q];
+              const T t = v[q];
               v[q] = v[q2];
               v[q2] = t;
             }
@@ -261,7 +269,7 @@ __device__ __forceinline__ void warp_sort_regs(uint64_t (&v)[V]) {
         const bool keep_min = ((lane & pl) == 0) == (((V * lane) & kk) == 0);
 #pragma unroll
         for (int q = 0; q < V; ++q) {
-          const uint64_t p = __shfl_xor_sync(0xffffffffu, v[q], pl);
+          const T p = __shfl_xor_sync(0xffffffffu, v[q], pl);
           v[q] = keep_min ? (v[q] < p ? v[q] : p) : (v[q] > p ? v[q] : p);
         }
       }

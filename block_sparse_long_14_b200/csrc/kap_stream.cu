@@ -46,14 +46,16 @@ namespace cosa {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kThreads = 480;
-constexpr int kQWarp = 0, kKWarp = 1, kPoolWarp0 = 2, kMmaWarp = 6, kEpiWarp0 = 7;
+constexpr int kThreads = 608;
+constexpr int kQWarp = 0, kKWarp = 1, kPoolWarp0 = 2, kMmaWarp = 10, kEpiWarp0 = 11;
 constexpr int kEpiThreads = 128;     // one epilogue group
 constexpr int kEpiBar0 = 2;          // named barriers 2 and 3: the two epilogue groups
+constexpr int kHeadBar0 = 4;         // named barriers 4 to 7: the two pooling warps of a head
 constexpr int kSelCap = 256;         // kept keys per row of the sampled selection
 constexpr int kRowWarps = 8;         // rows per CTA of the selection kernel
 constexpr int kKeys = 128;           // key blocks per score tile
 constexpr int kKStages = 3;
+constexpr int kAccBufs = 4;          // TMEM accumulators: two per epilogue group
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 __host__ __device__ constexpr int stream_np(int GT, int R) { return (GT * (R + 1) + 15) / 16 * 16; }
@@ -64,7 +66,7 @@ struct Shape {
   static constexpr int NP = stream_np(GT, R);      // MMA N (a multiple of 16)
   static constexpr int NS = GT * R;                // sub-rows of a tile
   static constexpr int ACC = NP <= 32 ? 32 : 64;   // TMEM columns per accumulator
-  static constexpr int TMEM_COLS = 4 * ACC;         // two accumulators per epilogue group
+  static constexpr int TMEM_COLS = kAccBufs * ACC;
   static constexpr int QSLOT = 16 * GT * kD * 2;   // one chunk: 16 rows x GT heads x d bf16
   static constexpr int KSLOT = kKeys * kD;         // one score tile of int8 key vectors
   static constexpr int ASLOT = NP * kD;            // the int8 query vectors (B operand)
@@ -75,7 +77,7 @@ struct Bars {
   uint64_t q_full[8], q_empty[8];
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t a_full[2], a_empty[2];
-  uint64_t acc_full[4], acc_empty[4];   // [2 group + buffer]
+  uint64_t acc_full[kAccBufs], acc_empty[kAccBufs];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -107,6 +109,134 @@ __device__ __forceinline__ uint32_t quantize4(const float (&x)[4], float& M_out)
   return packed;
 }
 
+// The epilogue group eg: takes the CTA's tiles of parity eg.  Each lane turns
+// one key block's dots into its score bits per head (written to the workspace
+// row of that head) and updates the sub-rows' running argmax; the group then
+// reduces the argmax to the HRM blocks of each head (written next to the
+// scores).
+template <int GT, int R>
+__device__ __forceinline__ void stream_epilogue(const ScoreArgs& a, const StreamLayout& lay, Bars* bars,
+                                                volatile int* abort, uint32_t tmem, unsigned char* smem) {
+  using S = Shape<GT, R>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int eg = (warp - kEpiWarp0) >> 2;
+  const int et = threadIdx.x - (kEpiWarp0 + 4 * eg) * 32;   // 0..127
+  const int ew = (warp - kEpiWarp0) & 3;
+  const int bar = kEpiBar0 + eg;
+  const int quad = warp & 3;                   // TMEM lane quadrant
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+  float* sKs = reinterpret_cast<float*>(smem + lay.ks + eg * lay.group_bytes);
+  uint64_t* red = reinterpret_cast<uint64_t*>(smem + lay.red + eg * lay.group_bytes);
+  const int ntiles = a.nqb_total * (a.num_q_heads / GT);
+  int u = 0, kloc = 0;   // key tiles consumed by this group; this CTA's good tiles so far
+  bool ok = true;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const Tile tl = tile_at<GT>(a, tile);
+    if (tl.bad || tl.npow2 > a.npow2_max) {
+      if (et == 0 && eg == 0) report(a.status, kErrBounds, 0x237);
+      continue;
+    }
+    if ((kloc++ & 1) != eg) continue;
+    const int n = tl.n;
+    const float* ks_row = a.ks + static_cast<long>(tl.kv) * a.nkb_total + tl.kb0;
+    for (int x = et; x < n; x += kEpiThreads) sKs[x] = __ldg(ks_row + x);
+    named_bar_sync(bar, kEpiThreads);
+    uint32_t* cand_row = a.cand + (static_cast<long>(tl.h0) * a.nqb_total + tl.I) * a.cand_stride;
+    const long cand_head = static_cast<long>(a.nqb_total) * a.cand_stride;   // one head further
+
+    // Each sub-row's best over this lane's key blocks: its score and the score tile it came
+    // from (8 bits each, four to a word).  The lane meets its blocks in ascending order, so a
+    // strictly higher score is needed to replace the best: on equal scores the lowest block
+    // stays, as in the packed order of pack_best.
+    float bs[S::NS];
+    uint32_t bk[(S::NS + 3) / 4];
+#pragma unroll
+    for (int x = 0; x < S::NS; ++x) bs[x] = -INFINITY;
+#pragma unroll
+    for (int x = 0; x < (S::NS + 3) / 4; ++x) bk[x] = 0u;
+    const int ntk = (n + kKeys - 1) / kKeys;
+    for (int kt = 0; kt < ntk; ++kt, ++u) {
+      const int ab = 2 * eg + (u & 1);
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->acc_full[ab], (u >> 1) & 1, kWaitLimit, abort,
+                                                   a.status, 0x238));
+      if (!ok) continue;
+      tc_fence_after();
+      const int j = kt * kKeys + 32 * quad + lane;         // this lane's key block
+      const float ksj = j < n ? sKs[j] : 0.0f;
+      // this lane's dots, 16 columns at a time: column mt (R + 1) is head mt's block
+      // vector (its score bits), the next R its sub-rows (their running argmax)
+#pragma unroll
+      for (int c = 0; c < S::NP / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(lane_base + ab * S::ACC + c * 16, r);
+        tc_wait_ld();
+        if (c == S::NP / 16 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);   // the accumulator may be overwritten
+        }
+        if (j < n) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = c * 16 + e;
+            if (col >= S::NV) continue;
+            const int mt = col / (R + 1), v = col % (R + 1);
+            const float sv = __fmul_rn(static_cast<float>(static_cast<int>(r[e])), ksj);
+            if (v == 0) {
+              cand_row[mt * cand_head + j] = score_bits(sv);
+            } else {
+              const int x = mt * R + v - 1;
+              if (sv > bs[x]) {
+                bs[x] = sv;
+                bk[x / 4] = bfi8(static_cast<uint32_t>(kt), bk[x / 4], 8 * (x % 4));
+              }
+            }
+          }
+        }
+      }
+    }
+    // each sub-row's best over the warp's 32 lanes by a butterfly that halves the entries a
+    // lane carries at each step (lane x ends with entry x), then over the group's four warps
+    uint64_t best[32];
+#pragma unroll
+    for (int x = 0; x < 32; ++x) {
+      if (x < S::NS) {
+        const int jx = 128 * static_cast<int>((bk[x / 4] >> (8 * (x % 4))) & 0xFFu) + 32 * quad + lane;
+        best[x] = bs[x] == -INFINITY ? 0ull : pack_best(bs[x], jx);
+      } else {
+        best[x] = 0ull;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int x = 0; x < o; ++x) {
+        const uint64_t send = upper ? best[x] : best[x + o];
+        const uint64_t keep = upper ? best[x + o] : best[x];
+        const uint64_t got = __shfl_xor_sync(0xffffffffu, send, o);
+        best[x] = got > keep ? got : keep;
+      }
+    }
+    if (lane < S::NS) red[ew * S::NS + lane] = best[0];
+    named_bar_sync(bar, kEpiThreads);
+    // the HRM blocks: each present sub-row's argmax (8 slots per head, -1 where none)
+    if (et < GT * 8 && ok) {
+      const int mt = et / 8, sr = et % 8;
+      int jv = -1;
+      if (sr < R) {
+        uint64_t v = red[mt * R + sr];
+#pragma unroll
+        for (int w = 1; w < 4; ++w) v = red[w * S::NS + mt * R + sr] > v ? red[w * S::NS + mt * R + sr] : v;
+        const int jj = static_cast<int>(~static_cast<uint32_t>(v));
+        if (v != 0ull && sub_present(tl, sr) && jj >= 0 && jj < n) jv = jj;
+      }
+      a.hrmj[((static_cast<long>(tl.h0 + mt) * a.nqb_total + tl.I) << 3) + sr] = jv;
+    }
+    named_bar_sync(bar, kEpiThreads);   // key scales and maxima are free for the group's next tile
+  }
+}
+
 }  // namespace
 
 template <int GT, int R>
@@ -122,9 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sQ = smem + lay.q;
   unsigned char* sK = smem + lay.k;
   unsigned char* sA = smem + lay.a;
-  // per epilogue group: key scales [npow2_max], sub-row maxima [4][NS]
-  float* sKs0 = reinterpret_cast<float*>(smem + lay.ks);
-  uint64_t* red0 = reinterpret_cast<uint64_t*>(smem + lay.red);
+  float* sSub = reinterpret_cast<float*>(smem + lay.sub);
   Bars* bars = reinterpret_cast<Bars*>(smem + lay.bars);
   volatile int* abort = &bars->abort;
   const int QS = lay.q_stages;
@@ -137,17 +265,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (a.retry != nullptr && blockIdx.x == 0) a.retry[0] = 0;   // the selection's retry list starts empty
     for (int x = 0; x < QS; ++x) {
       mbar_init(&bars->q_full[x], 1);
-      mbar_init(&bars->q_empty[x], 4);            // the four pooling warps
+      mbar_init(&bars->q_empty[x], 4);            // the four pooling warps of the chunk's parity
     }
     for (int x = 0; x < kKStages; ++x) {
       mbar_init(&bars->k_full[x], 1);
       mbar_init(&bars->k_empty[x], 1);
     }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&bars->a_full[x], 4);             // the four pooling warps
+      mbar_init(&bars->a_full[x], 8);             // the eight pooling warps
       mbar_init(&bars->a_empty[x], 1);
     }
-    for (int x = 0; x < 4; ++x) {
+    for (int x = 0; x < kAccBufs; ++x) {
       mbar_init(&bars->acc_full[x], 1);
       mbar_init(&bars->acc_empty[x], 4);          // the four warps of the group
     }
@@ -215,8 +343,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = max(0, kc - kKStages); c < kc; ++c) mbar_drain(&bars->k_full[c % kKStages], (c / kKStages) & 1);
     }
   } else if (warp < kMmaWarp) {
-    // ======================================================== pooling (one query head per warp)
+    // ======================================================== pooling: two warps per query head,
+    // the even and the odd sub-rows
     const int pw = warp - kPoolWarp0;
+    const int mt = pw & 3, half = pw >> 2;
+    const bool active = mt < GT;
     int qc = 0, tcount = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -227,15 +358,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->a_empty[buf], ((tcount >> 1) - 1) & 1, kWaitLimit,
                                                      abort, a.status, 0x232));
       unsigned char* amat = sA + buf * S::ASLOT;
-      float blk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      for (int v = 0; v < R; ++v, ++qc) {
-        const int slot = qc % QS;
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->q_full[slot], (qc / QS) & 1, kWaitLimit, abort,
+      // the sub-row sums of head mt go through shared memory (double-buffered across tiles)
+      float* sums = sSub + (buf * GT + (active ? mt : 0)) * R * kD + lane * 4;
+#pragma unroll 1
+      for (int v = half; v < R; v += 2) {
+        const int c = qc + v, slot = c % QS;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->q_full[slot], (c / QS) & 1, kWaitLimit, abort,
                                                      a.status, 0x233));
-        if (ok && pw < GT) {
+        if (ok && active) {
           // sub-row v: rows 16v .. 16v + 15 of the tile, summed token by token (present rows
           // only); all 16 rows are read first so the loads overlap
-          const unsigned char* src = sQ + slot * S::QSLOT + pw * (kD * 2) + lane * 8;
+          const unsigned char* src = sQ + slot * S::QSLOT + mt * (kD * 2) + lane * 8;
           uint2 raw[16];
 #pragma unroll
           for (int rr = 0; rr < 16; ++rr) raw[rr] = *reinterpret_cast<const uint2*>(src + rr * (GT * kD * 2));
@@ -250,20 +383,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               sub[3] = __fadd_rn(sub[3], __uint_as_float(raw[rr].y & 0xFFFF0000u));
             }
           }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) blk[e] = __fadd_rn(blk[e], sub[e]);   // the q-block sum: their fold
+          *reinterpret_cast<float4*>(sums + v * kD) = make_float4(sub[0], sub[1], sub[2], sub[3]);
           float M;
           const uint32_t packed = quantize4(sub, M);
-          store_vec(amat, pw * (R + 1) + 1 + v, lane, packed);
+          store_vec(amat, mt * (R + 1) + 1 + v, lane, packed);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_empty[slot]);
       }
-      if (ok && pw < GT) {
+      qc += R;
+      // the q-block vector: the fold of the sub-row sums in order (their sum from zero), by the
+      // even warp once the odd one has written its sums
+      named_bar_sync(kHeadBar0 + mt, 64);
+      if (ok && active && half == 0) {
+        float blk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int v = 0; v < R; ++v) {
+          const float4 t = *reinterpret_cast<const float4*>(sums + v * kD);
+          blk[0] = __fadd_rn(blk[0], t.x);
+          blk[1] = __fadd_rn(blk[1], t.y);
+          blk[2] = __fadd_rn(blk[2], t.z);
+          blk[3] = __fadd_rn(blk[3], t.w);
+        }
         float M;
         const uint32_t packed = quantize4(blk, M);
-        store_vec(amat, pw * (R + 1), lane, packed);
-        if (a.qm != nullptr && lane == 0) a.qm[static_cast<long>(tl.h0 + pw) * a.nqb_total + tl.I] = M;
+        store_vec(amat, mt * (R + 1), lane, packed);
+        if (a.qm != nullptr && lane == 0) a.qm[static_cast<long>(tl.h0 + mt) * a.nqb_total + tl.I] = M;
       }
       fence_proxy_async();   // the generic-proxy stores reach the tensor core's view of shared memory
       __syncwarp();
@@ -312,98 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ======================================================== epilogue: scores and HRM flags
-    const int eg = (warp - kEpiWarp0) >> 2;      // epilogue group: takes the CTA's tiles of parity eg
-    const int et = tid - (kEpiWarp0 + 4 * eg) * 32;   // 0..127
-    const int ew = (warp - kEpiWarp0) & 3;
-    const int bar = kEpiBar0 + eg;
-    const int quad = warp & 3;                   // TMEM lane quadrant
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quad) << 16);
-    float* sKs = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(sKs0) + eg * lay.group_bytes);
-    uint64_t* red = red0 + eg * (lay.group_bytes / 8);
-    int u = 0, kloc = 0;   // key tiles consumed by this group; this CTA's good tiles so far
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-      const Tile tl = tile_at<GT>(a, tile);
-      if (tl.bad || tl.npow2 > a.npow2_max) {
-        if (et == 0 && eg == 0) report(a.status, kErrBounds, 0x237);
-        continue;
-      }
-      if ((kloc++ & 1) != eg) continue;
-      const int n = tl.n;
-      const float* ks_row = a.ks + static_cast<long>(tl.kv) * a.nkb_total + tl.kb0;
-      for (int x = et; x < n; x += kEpiThreads) sKs[x] = __ldg(ks_row + x);
-      named_bar_sync(bar, kEpiThreads);
-      uint32_t* cand_row = a.cand + (static_cast<long>(tl.h0) * a.nqb_total + tl.I) * a.cand_stride;
-      const long cand_head = static_cast<long>(a.nqb_total) * a.cand_stride;   // one head further
-
-      uint64_t best[S::NS];
-#pragma unroll
-      for (int x = 0; x < S::NS; ++x) best[x] = 0ull;
-      const int ntk = (n + kKeys - 1) / kKeys;
-      for (int kt = 0; kt < ntk; ++kt, ++u) {
-        const int ab = 2 * eg + (u & 1);
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->acc_full[ab], (u >> 1) & 1, kWaitLimit, abort,
-                                                     a.status, 0x238));
-        if (!ok) continue;
-        tc_fence_after();
-        const int j = kt * kKeys + 32 * quad + lane;         // this lane's key block
-        const float ksj = j < n ? sKs[j] : 0.0f;
-        // this lane's dots, 16 columns at a time: column mt (R + 1) is head mt's block
-        // vector (its score bits), the next R its sub-rows (their running argmax)
-#pragma unroll
-        for (int c = 0; c < S::NP / 16; ++c) {
-          uint32_t r[16];
-          tmem_ld16(lane_base + ab * S::ACC + c * 16, r);
-          tc_wait_ld();
-          if (c == S::NP / 16 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);   // the accumulator may be overwritten
-          }
-          if (j < n) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int col = c * 16 + e;
-              if (col >= S::NV) continue;
-              const int mt = col / (R + 1), v = col % (R + 1);
-              const float sv = __fmul_rn(static_cast<float>(static_cast<int>(r[e])), ksj);
-              if (v == 0) {
-                cand_row[mt * cand_head + j] = score_bits(sv);
-              } else {
-                const uint64_t cand = pack_best(sv, j);
-                if (cand > best[mt * R + v - 1]) best[mt * R + v - 1] = cand;
-              }
-            }
-          }
-        }
-      }
-      // each sub-row's best over the warp's 32 lanes, then over the group's four warps
-#pragma unroll
-      for (int x = 0; x < S::NS; ++x) {
-        uint64_t v = best[x];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
-          v = o > v ? o : v;
-        }
-        if (lane == 0) red[ew * S::NS + x] = v;
-      }
-      named_bar_sync(bar, kEpiThreads);
-      // the HRM blocks: each present sub-row's argmax (8 slots per head, -1 where none)
-      if (et < GT * 8 && ok) {
-        const int mt = et / 8, sr = et % 8;
-        int jv = -1;
-        if (sr < R) {
-          uint64_t v = red[mt * R + sr];
-#pragma unroll
-          for (int w = 1; w < 4; ++w) v = red[w * S::NS + mt * R + sr] > v ? red[w * S::NS + mt * R + sr] : v;
-          const int jj = static_cast<int>(~static_cast<uint32_t>(v));
-          if (v != 0ull && sub_present(tl, sr) && jj >= 0 && jj < n) jv = jj;
-        }
-        a.hrmj[((static_cast<long>(tl.h0 + mt) * a.nqb_total + tl.I) << 3) + sr] = jv;
-      }
-      named_bar_sync(bar, kEpiThreads);   // key scales and maxima are free for the group's next tile
-    }
+    stream_epilogue<GT, R>(a, lay, bars, abort, tmem, smem);
   }
 
   tc_fence_before();
@@ -517,10 +571,11 @@ __global__ void __launch_bounds__(kRowWarps * 32) select_rows_kernel(const Score
 // One warp per row, longest rows first, with no per-row shared-memory copy of
 // the keys: each key is rebuilt from the row's score bits (read from L2, where
 // the score kernel left them) and the row's HRM blocks (held in every lane).
-// Rows of at most 128 candidates are sorted whole in registers; longer rows
-// take a sampled threshold (64 keys at evenly spaced positions, sorted in
-// registers), one ballot pass that compacts the keys at or below it into a
-// 256-key buffer, and a register sort of the kept set.  A row whose kept set
+// Rows of at most 32 candidates (or whose budget keeps them all) are sorted
+// whole in registers; longer rows take a sampled threshold (the upper 32 bits
+// of 64 keys at evenly spaced positions, sorted in registers), one ballot pass
+// that compacts the keys at or below it into a 256-key buffer, and a register
+// sort of the kept set (32, 64, 128 or 256 keys wide).  A row whose kept set
 // does not fit, or whose samples never reach k_i, goes to the retry list
 // (list[0] = length, list[1..] = rows) that select_rows_kernel finishes.
 constexpr int kFastWarps = 8;
@@ -528,13 +583,27 @@ constexpr int kFastCap = 256;
 
 struct RowKeys {
   const uint32_t* cr;
-  int hb[8];   // the row's HRM blocks (-1: none)
+  int hb[8];        // the row's HRM blocks (-1: none)
+  uint64_t lmask;   // bit m: block 32 m + lane is an HRM block (m < 64)
+  __device__ __forceinline__ void init(int lane) {
+    lmask = 0ull;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (hb[q] >= 0 && (hb[q] & 31) == lane && hb[q] < 64 * 32) lmask |= 1ull << (hb[q] >> 5);
+  }
+  // the sort key of block x
   __device__ __forceinline__ uint64_t at(int x) const {
     const uint64_t key = key_of(__ldg(cr + x), x);
     bool f = false;
 #pragma unroll
     for (int q = 0; q < 8; ++q) f |= hb[q] == x;
     return f ? key & ~(1ull << 63) : key;
+  }
+  // the same for a block of this lane (x = 32 m + lane)
+  __device__ __forceinline__ uint64_t at_lane(int x) const {
+    if (x >= 64 * 32) return at(x);
+    const uint64_t key = key_of(__ldg(cr + x), x);
+    return ((lmask >> (x >> 5)) & 1ull) ? key & ~(1ull << 63) : key;
   }
 };
 
@@ -574,8 +643,9 @@ __device__ __forceinline__ void sort_emit(const ScoreArgs& a, long row, const Ro
   uint64_t v[V];
 #pragma unroll
   for (int q = 0; q < V; ++q) {
-    const int e = V * lane + q;
-    v[q] = e < cnt ? (buf != nullptr ? buf[e] : rk.at(e)) : ~0ull;
+    // any placement before the sort: the row's own blocks by lane, the buffer's in runs
+    const int x = buf != nullptr ? V * lane + q : 32 * q + lane;
+    v[q] = x < cnt ? (buf != nullptr ? buf[x] : rk.at_lane(x)) : ~0ull;
   }
   warp_sort_regs<V>(v);
   emit_row<V>(a, row, v, k_out);
@@ -603,53 +673,63 @@ __global__ void __launch_bounds__(kFastWarps * 32) select_fast_kernel(const Scor
   const int hj = lane < 8 ? __ldg(a.hrmj + row * 8 + lane) : -1;
 #pragma unroll
   for (int q = 0; q < 8; ++q) rk.hb[q] = __shfl_sync(kFull, hj, q);
+  rk.init(lane);
   const int k_i = keep_count(n, a.bp);
   const int k_out = min(k_i, a.kmax);
   if (k_out < k_i && lane == 0) report(a.status, kErrBounds, 0x245);   // host sizing forbids it
 
-  if (n <= 64) {
-    sort_emit<2>(a, row, rk, nullptr, n, k_out);
+  if (k_i == n || n <= 32) {
+    // every candidate kept, or few: sort them all
+    if (n <= 32) sort_emit<1>(a, row, rk, nullptr, n, k_out);
+    else if (n <= 64) sort_emit<2>(a, row, rk, nullptr, n, k_out);
+    else if (n <= 128) sort_emit<4>(a, row, rk, nullptr, n, k_out);
+    else if (n <= 256) sort_emit<8>(a, row, rk, nullptr, n, k_out);
+    else if (lane == 0) a.retry[1 + atomicAdd(a.retry, 1)] = static_cast<int32_t>(rr);
     return;
   }
-  if (n <= 128) {
-    sort_emit<4>(a, row, rk, nullptr, n, k_out);
-    return;
-  }
-  int cnt = -1;
-  if (k_i < n) {
-    // sample element e = 2 lane + q, taken at position (e n) / 64
-    uint64_t smp[2] = {rk.at((2 * lane * n) >> 6), rk.at(((2 * lane + 1) * n) >> 6)};
-    warp_sort_regs<2>(smp);
-    int r = min(63, (64 * k_i + n - 1) / n + 1);   // about 2 k_i keys at or below the r-th sample
-    for (int attempt = 0; attempt < 3; ++attempt) {
-      const uint64_t t0 = __shfl_sync(kFull, smp[0], r >> 1), t1 = __shfl_sync(kFull, smp[1], r >> 1);
-      const uint64_t T = (r & 1) ? t1 : t0;
-      cnt = 0;
-      for (int base = 0; base < n; base += 128) {   // four loads in flight per lane
-        uint64_t key[4];
+  // The threshold compares the keys' upper 32 bits (flag and score bits but the lowest):
+  // the keys kept form a down-set of the order, so once there are k_i of them they hold the
+  // k_i smallest.  Sample element e = 2 lane + q, taken at position (e n) / 64.
+  uint32_t smp[2] = {static_cast<uint32_t>(rk.at((2 * lane * n) >> 6) >> 32),
+                     static_cast<uint32_t>(rk.at(((2 * lane + 1) * n) >> 6) >> 32)};
+  warp_sort_regs<2>(smp);
+  int r = min(63, (64 * k_i + n - 1) / n + 1);   // about 2 k_i keys at or below the r-th sample
+  int cnt = 0;
+  for (int attempt = 0; attempt < 3; ++attempt) {
+    const uint32_t t0 = __shfl_sync(kFull, smp[0], r >> 1), t1 = __shfl_sync(kFull, smp[1], r >> 1);
+    const uint32_t T = (r & 1) ? t1 : t0;
+    cnt = 0;
+    for (int base = 0; base < n; base += 128) {   // four loads in flight per lane
+      uint64_t key[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int x = base + 32 * u + lane;
-          key[u] = x < n ? rk.at(x) : ~0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const bool keep = base + 32 * u + lane < n && key[u] <= T;
-          const unsigned bal = __ballot_sync(kFull, keep);
-          const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-          if (keep && pos < kFastCap) buf[pos] = key[u];
-          cnt += __popc(bal);
-        }
+      for (int u = 0; u < 4; ++u) {
+        const int x = base + 32 * u + lane;
+        key[u] = x < n ? rk.at_lane(x) : ~0ull;
       }
-      if (cnt >= k_i || r == 63) break;
-      r = min(63, r + r / 2 + 2);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool keep = base + 32 * u + lane < n && static_cast<uint32_t>(key[u] >> 32) <= T;
+        const unsigned bal = __ballot_sync(kFull, keep);
+        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        if (keep && pos < kFastCap) buf[pos] = key[u];
+        cnt += __popc(bal);
+      }
     }
-    __syncwarp();
+    if (cnt >= k_i || r == 63) break;
+    r = min(63, r + r / 2 + 2);
   }
-  if (cnt >= k_i && cnt <= 64) sort_emit<2>(a, row, rk, buf, cnt, k_out);
-  else if (cnt >= k_i && cnt <= 128) sort_emit<4>(a, row, rk, buf, cnt, k_out);
-  else if (cnt >= k_i && cnt <= kFastCap) sort_emit<8>(a, row, rk, buf, cnt, k_out);
-  else if (lane == 0) a.retry[1 + atomicAdd(a.retry, 1)] = static_cast<int32_t>(rr);
+  __syncwarp();
+  if (cnt < k_i || cnt > kFastCap) {
+    if (lane == 0) a.retry[1 + atomicAdd(a.retry, 1)] = static_cast<int32_t>(rr);
+  } else if (cnt <= 32) {
+    sort_emit<1>(a, row, rk, buf, cnt, k_out);
+  } else if (cnt <= 64) {
+    sort_emit<2>(a, row, rk, buf, cnt, k_out);
+  } else if (cnt <= 128) {
+    sort_emit<4>(a, row, rk, buf, cnt, k_out);
+  } else {
+    sort_emit<8>(a, row, rk, buf, cnt, k_out);
+  }
 }
 
 // ============================================================ host side
@@ -665,6 +745,8 @@ StreamLayout stream_layout(int GT, int R, int npow2_max, int kmax, int q_stages)
   off += kKStages * kKeys * kD;
   L.a = off;
   off += 2 * np * kD;
+  L.sub = off;
+  off += 2 * GT * R * kD * 4;
   // one region per epilogue group: key scales, sub-row maxima
   uint32_t g = 0;
   L.ks = off + g;
@@ -680,7 +762,11 @@ StreamLayout stream_layout(int GT, int R, int npow2_max, int kmax, int q_stages)
 }
 
 bool stream_fits(int GT, int R, int npow2_max, int kmax, int* q_stages) {
-  for (int qs = 6; qs >= 3; --qs) {
+  // an even ring: chunk c goes to slot c % QS and to the pooling warps of parity c % 2, so
+  // each slot serves one parity and its waits come in order (with an odd ring the
+  // even-chunk warps could wait on a slot's next use before its current chunk landed,
+  // where the phase parity cannot tell the two apart)
+  for (int qs = 8; qs >= 4; qs -= 2) {
     if (stream_layout(GT, R, npow2_max, kmax, qs).total <= kStreamSmemLimit) {
       *q_stages = qs;
       return true;

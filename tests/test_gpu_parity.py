@@ -376,7 +376,8 @@ def _sample_defeating_workload():
     s_j.  For the last q-block (n = 512) the 64 threshold samples of the
     register selection sit at blocks 8e.  Kv head 0 gives those 64 blocks the
     highest scores: at a 5 % budget (k = 26) no sample rank tried (the 6th,
-    10th and 16th smallest) has k keys at or below it.  Kv head 1 gives them
+    10th and 16th smallest) has k keys at or below it (nor within the
+    threshold's lowest score bit of it).  Kv head 1 gives them
     the lowest scores: every sample has more than the 256 keys the kept buffer
     holds below it.  Both rows must finish in the shared-memory selection."""
     from synth import from_arrays
@@ -386,8 +387,8 @@ def _sample_defeating_workload():
     u = np.ones(d, dtype=np.float32) / np.sqrt(d)
     on = np.zeros(nb, dtype=bool)
     on[::8] = True
-    hi = 2.0 + 0.5 * rng.random(nb)
-    lo = -1.0 - 0.5 * rng.random(nb)
+    hi = 2.0 + 6.0 * rng.random(nb)    # few equal bf16 values among the 64 sampled blocks
+    lo = -1.0 - 6.0 * rng.random(nb)
     s = np.stack([np.where(on, hi, lo), np.where(on, -hi, -lo)], axis=1)   # [nb, kv head]
     k = np.repeat(s, b, axis=0)[:, :, None] * u[None, None, :]
     q = np.broadcast_to(u, (L, 2, d)).astype(np.float32)

@@ -1,19 +1,20 @@
 """The mbarrier protocol of the persistent proxy kernel (kap_stream.cu), simulated on the CPU.
 
 The kernel's roles hand work to each other through mbarriers: the Q producer
-fills a ring of QS chunk slots (q_full / q_empty, four pooling warps release
-a slot); the key producer fills a ring of 3 key-tile slots (k_full / k_empty,
-released by the MMAs' commit); the four pooling warps fill one of two B-operand
-buffers per tile (a_full, four arrivals; a_empty, the MMAs' commit after the
-tile's last key tile); two epilogue groups of four warps take alternate
-tiles, and the MMA issuer fills, for each key tile, one of the two TMEM
-accumulators of the tile's group (acc_full by commit; acc_empty, the group's
-four warps); a group's warps meet at its named barrier between the phases of
-a tile.  This model
-replays each role's waits (with the kernel's parities) and arrivals over a
-CTA's sequence of tiles with random key-tile counts, with copies and MMAs
-completing asynchronously (MMAs in issue order).  Every run must complete,
-and each wait must be satisfied by exactly the phase it intends.
+fills a ring of QS chunk slots (q_full / q_empty; the four pooling warps of
+the chunk's parity release a slot); the key producer fills a ring of 3
+key-tile slots (k_full / k_empty, released by the MMAs' commit); eight pooling
+warps (two per head: the even and the odd sub-rows, meeting at the head's
+named barrier before the block vector) fill one of two B-operand buffers per
+tile (a_full, eight arrivals; a_empty, the MMAs' commit after the tile's last
+key tile); two epilogue groups of four warps take alternate tiles, and the
+MMA issuer fills, for each key tile, one of the two TMEM accumulators of the
+tile's group (acc_full by commit; acc_empty, the group's four warps); a
+group's warps meet at its named barrier between the phases of a tile.  This
+model replays each role's waits (with the kernel's parities) and arrivals
+over a CTA's sequence of tiles with random key-tile counts, with copies and
+MMAs completing asynchronously (MMAs in issue order).  Every run must
+complete, and each wait must be satisfied by exactly the phase it intends.
 """
 import random
 
@@ -42,7 +43,7 @@ class Bar:
 
 
 class NamedBarrier:
-    """bar.sync among the four epilogue warps: generation counter."""
+    """bar.sync among n warps: generation counter."""
 
     def __init__(self, n):
         self.n, self.waiting, self.gen = n, 0, 0
@@ -63,10 +64,11 @@ def run(ntk, R, QS, rng):
     q_empty = [Bar(4) for _ in range(QS)]
     k_full = [Bar(1) for _ in range(KS)]
     k_empty = [Bar(1) for _ in range(KS)]
-    a_full, a_empty = [Bar(4), Bar(4)], [Bar(1), Bar(1)]
+    a_full, a_empty = [Bar(8), Bar(8)], [Bar(1), Bar(1)]
     acc_full, acc_empty = [Bar(1) for _ in range(4)], [Bar(4) for _ in range(4)]   # [2 group + buffer]
     drain = Bar(1)
     epi_bar = [NamedBarrier(4), NamedBarrier(4)]
+    head_bar = [NamedBarrier(2) for _ in range(4)]
     pending = []                        # async completions, ('copy', bar) or ('mma', [bars])
 
     def q_producer():
@@ -97,21 +99,25 @@ def run(ntk, R, QS, rng):
             while not k_full[c % KS].ready((c // KS) & 1, c // KS):
                 yield
 
-    def pooling():
+    def pooling(mt, half):
         qc = 0
         for tcount, _ in enumerate(ntk):
             buf = tcount & 1
             if tcount >= 2:
                 while not a_empty[buf].ready(((tcount >> 1) - 1) & 1, (tcount >> 1) - 1):
                     yield
-            for _v in range(R):
-                slot = qc % QS
-                while not q_full[slot].ready((qc // QS) & 1, qc // QS):
+            for v in range(R):
+                if (v & 1) != half:
+                    continue
+                c = qc + v
+                slot = c % QS
+                while not q_full[slot].ready((c // QS) & 1, c // QS):
                     yield
                 yield                                           # sums the chunk, writes the vector
                 q_empty[slot].arrive()
-                qc += 1
-            yield                                               # the block vector
+            qc += R
+            yield from head_bar[mt].sync()                      # the odd sums are written
+            yield                                               # the block vector (even warp)
             a_full[buf].arrive()
 
     def mma():
@@ -156,7 +162,7 @@ def run(ntk, R, QS, rng):
             yield                                               # HRM blocks written
             yield from epi_bar[eg].sync()                       # scales and maxima free for the next tile
 
-    alive = ([q_producer(), k_producer(), mma()] + [pooling() for _ in range(4)] +
+    alive = ([q_producer(), k_producer(), mma()] + [pooling(mt, half) for half in (0, 1) for mt in range(4)] +
              [epilogue(eg) for eg in (0, 1) for _ in range(4)])
     steps = 0
     while alive or pending:
@@ -177,7 +183,7 @@ def run(ntk, R, QS, rng):
             alive.remove(r)
 
 
-@pytest.mark.parametrize("QS", [3, 4, 6])
+@pytest.mark.parametrize("QS", [4, 6, 8])
 @pytest.mark.parametrize("R", [4, 8])
 def test_proxy_stream_protocol_completes_on_its_intended_phases(QS, R):
     rng = random.Random(QS * 10 + R)
@@ -192,9 +198,20 @@ def test_a_wrong_parity_is_caught():
     import inspect
     src = inspect.getsource(run).replace("acc_empty[ab].ready(((u >> 1) - 1) & 1",
                                          "acc_empty[ab].ready((u >> 1) & 1")
+    assert src != inspect.getsource(run)
     ns = dict(globals())
     exec(compile(src, "mutant", "exec"), ns)
     with pytest.raises(AssertionError):
         rng = random.Random(0)
         for _ in range(20):
             ns["run"]([3, 5, 2, 7], 8, 4, rng)
+
+
+def test_an_odd_q_ring_is_caught():
+    """With an odd ring a slot serves both parities in turn, and the even-chunk warps can
+    wait on a slot's next use before the odd warps' chunk in it has landed: the model
+    reports the aliased phase (the kernel takes an even ring only)."""
+    with pytest.raises(AssertionError):
+        rng = random.Random(1)
+        for _ in range(40):
+            run([rng.randint(1, 9) for _ in range(5)], 8, 3, rng)
