@@ -101,10 +101,11 @@ size_t select_tc_smem_bytes(int GT, int npow2_max, int scratch_bytes);
 // The persistent proxy kernel (head_dim 128, budget cut): pooling, scores and
 // HRM flags of every tile in one launch, one CTA per SM, writing a.cand and
 // a.hrmj.  Shared-memory layout (byte offsets from a 1024-aligned base: Q
-// ring, key tiles, int8 query vectors, odd sub-row sums; ks and red are those
-// of epilogue group 0, group 1's follow group_bytes later) and its limit:
+// ring, key tiles, int8 query vectors, sub-row sums, tile table; ks and red
+// are those of epilogue group 0, group 1's follow group_bytes later) and its
+// limit:
 struct StreamLayout {
-  uint32_t q, k, a, sub, ks, red, group_bytes, bars, total;
+  uint32_t q, k, a, sub, tiles, ks, red, group_bytes, bars, total;
   int q_stages;   // Q chunks in flight (16 rows each)
 };
 constexpr uint32_t kStreamSmemLimit = 227 * 1024;

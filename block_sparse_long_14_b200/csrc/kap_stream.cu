@@ -109,6 +109,17 @@ __device__ __forceinline__ uint32_t quantize4(const float (&x)[4], float& M_out)
   return packed;
 }
 
+// The CTA's first kTileCache tiles are described once, in the prologue, into
+// shared memory; every role reads them from there (later tiles, if any, are
+// described where they are met).
+constexpr int kTileCache = 64;
+
+template <int GT>
+__device__ __forceinline__ Tile cached_tile(const ScoreArgs& a, const Tile* tiles, int tile) {
+  const int it = (tile - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
+  return it < kTileCache ? tiles[it] : tile_at<GT>(a, tile);
+}
+
 // The epilogue group eg: takes the CTA's tiles of parity eg.  Each lane turns
 // one key block's dots into its score bits per head (written to the workspace
 // row of that head) and updates the sub-rows' running argmax; the group then
@@ -116,7 +127,8 @@ __device__ __forceinline__ uint32_t quantize4(const float (&x)[4], float& M_out)
 // scores).
 template <int GT, int R>
 __device__ __forceinline__ void stream_epilogue(const ScoreArgs& a, const StreamLayout& lay, Bars* bars,
-                                                volatile int* abort, uint32_t tmem, unsigned char* smem) {
+                                                volatile int* abort, uint32_t tmem, unsigned char* smem,
+                                                const Tile* tiles) {
   using S = Shape<GT, R>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int eg = (warp - kEpiWarp0) >> 2;
@@ -131,7 +143,7 @@ __device__ __forceinline__ void stream_epilogue(const ScoreArgs& a, const Stream
   int u = 0, kloc = 0;   // key tiles consumed by this group; this CTA's good tiles so far
   bool ok = true;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const Tile tl = tile_at<GT>(a, tile);
+    const Tile tl = cached_tile<GT>(a, tiles, tile);
     if (tl.bad || tl.npow2 > a.npow2_max) {
       if (et == 0 && eg == 0) report(a.status, kErrBounds, 0x237);
       continue;
@@ -253,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sK = smem + lay.k;
   unsigned char* sA = smem + lay.a;
   float* sSub = reinterpret_cast<float*>(smem + lay.sub);
+  Tile* tiles = reinterpret_cast<Tile*>(smem + lay.tiles);
   Bars* bars = reinterpret_cast<Bars*>(smem + lay.bars);
   volatile int* abort = &bars->abort;
   const int QS = lay.q_stages;
@@ -283,6 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort = 0;
     mbar_fence_init();
   }
+  for (int x = tid; x < kTileCache; x += kThreads) {
+    const int tile = blockIdx.x + x * gridDim.x;
+    if (tile < ntiles) tiles[x] = tile_at<GT>(a, tile);
+  }
   // the padding rows of both B-operand buffers stay zero
   for (int x = tid; x < 2 * (S::NP - S::NV) * 32; x += kThreads) {
     const int buf = x / ((S::NP - S::NV) * 32), rem = x % ((S::NP - S::NV) * 32);
@@ -305,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int qc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const Tile tl = tile_at<GT>(a, tile);
+        const Tile tl = cached_tile<GT>(a, tiles, tile);
         if (tl.bad || tl.npow2 > a.npow2_max) continue;
         for (int v = 0; v < R && ok; ++v, ++qc) {
           const int slot = qc % QS, use = qc / QS;
@@ -327,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int kc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const Tile tl = tile_at<GT>(a, tile);
+        const Tile tl = cached_tile<GT>(a, tiles, tile);
         if (tl.bad || tl.npow2 > a.npow2_max) continue;
         const int ntk = (tl.n + kKeys - 1) / kKeys;
         const int row0 = tl.kv * a.nkb_total + tl.kb0;
@@ -351,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int qc = 0, tcount = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-      const Tile tl = tile_at<GT>(a, tile);
+      const Tile tl = cached_tile<GT>(a, tiles, tile);
       if (tl.bad || tl.npow2 > a.npow2_max) continue;
       const int buf = tcount & 1;
       if (tcount >= 2)
@@ -422,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int accg[2] = {0, 0};   // key tiles issued to each epilogue group
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const Tile tl = tile_at<GT>(a, tile);
+        const Tile tl = cached_tile<GT>(a, tiles, tile);
         if (tl.bad || tl.npow2 > a.npow2_max) continue;
         const int buf = tcount & 1, eg = tcount & 1;   // the tile's B-operand buffer and epilogue group
         ok = mbar_wait(&bars->a_full[buf], (tcount >> 1) & 1, kWaitLimit, abort, a.status, 0x234);
@@ -457,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ======================================================== epilogue: scores and HRM flags
-    stream_epilogue<GT, R>(a, lay, bars, abort, tmem, smem);
+    stream_epilogue<GT, R>(a, lay, bars, abort, tmem, smem, tiles);
   }
 
   tc_fence_before();
@@ -747,6 +764,8 @@ StreamLayout stream_layout(int GT, int R, int npow2_max, int kmax, int q_stages)
   off += 2 * np * kD;
   L.sub = off;
   off += 2 * GT * R * kD * 4;
+  L.tiles = off;
+  off += (kTileCache * sizeof(Tile) + 15) / 16 * 16;
   // one region per epilogue group: key scales, sub-row maxima
   uint32_t g = 0;
   L.ks = off + g;
