@@ -64,6 +64,16 @@ def tensor_peak(pk, clocks):
                                 f"{mhz:.0f} / {pk['sm_max_mhz']:.0f} MHz")
 
 
+def proxy_kernels(w, kmax):
+    """The kernels one budget-cut proxy call launches: at head_dim 128 the
+    persistent scoring kernel and the register selection (its retry pass always
+    launches; kmax <= 128), else the two-stage pool / select kernels."""
+    if w.head_dim == 128:
+        return ["kpool", "kap_stream", "select_fast", "select_rows"] if kmax <= 128 else \
+               ["kpool", "kap_stream", "select_rows"]
+    return ["kpool", "qpool", "kap_select"]
+
+
 def measured_traffic():
     """DRAM bytes per OSK launch from the committed ncu launch list, or None
     when the kernel's sources changed since those counters were taken."""
@@ -647,9 +657,9 @@ def run_cosa(args, rank, world, local_rank):
                      "algorithmic": f"{exec_flops:.4e} FLOP per launch = 2*128*128*128 * (visited + kept)"},
         "proxy_roofline": {"bound": "hbm", "achieved": proxy_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                            "frac": proxy_gbs / pk["hbm_gbs"], "algorithmic_bytes": proxy_bytes,
-                           "kernels": "kpool + qpool + kap_select_tc"},
+                           "kernels": " + ".join(proxy_kernels(w, kmax))},
         "clocks": clocks,
-        "gpu_launches": 4 * args.steps,   # kpool, qpool, select, osk per step
+        "gpu_launches": (len(proxy_kernels(w, kmax)) + 1) * args.steps,   # the proxy's kernels and osk per step
         "e2e": e2e,
         **extra,
     }
