@@ -290,6 +290,7 @@ int proxy_impl(const cosa_shape_t* shape, const void* q, const void* k_pages, co
     sa.hrmj = reinterpret_cast<int32_t*>(ws + w.hrmj_off);
     sa.cand_stride = w.cand_stride;
     sa.retry = reinterpret_cast<int32_t*>(ws + w.retry_off);
+    sa.wait_limit = g_wait_limit.load();
     const StreamLayout lay = stream_layout(GT, shape->block_size / 16, sa.npow2_max, kmax, q_stages);
     if (launch_stream(sa, GT, q_map, kq_map, lay, st) != cudaSuccess) return COSA_ERR_CUDA;
     return launch_select_rows(sa, st) == cudaSuccess ? COSA_OK : COSA_ERR_CUDA;

@@ -50,6 +50,7 @@ struct ScoreArgs {
   int cand_stride;     // candidates per row the cand rows hold (the longest sequence's key blocks)
   int32_t* retry;      // [1 + Hq * NQB] rows the register selection leaves to select_rows_kernel
                        // (retry[0] = how many; nullable: every row by select_rows_kernel)
+  uint32_t wait_limit; // polls per mbarrier wait of the persistent proxy kernel
 };
 
 struct RemapArgs {

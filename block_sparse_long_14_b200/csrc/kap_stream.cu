@@ -56,7 +56,6 @@ constexpr int kRowWarps = 8;         // rows per CTA of the selection kernel
 constexpr int kKeys = 128;           // key blocks per score tile
 constexpr int kKStages = 3;
 constexpr int kAccBufs = 4;          // TMEM accumulators: two per epilogue group
-constexpr uint32_t kWaitLimit = 1u << 22;
 
 __host__ __device__ constexpr int stream_np(int GT, int R) { return (GT * (R + 1) + 15) / 16 * 16; }
 
@@ -169,7 +168,7 @@ __device__ __forceinline__ void stream_epilogue(const ScoreArgs& a, const Stream
     const int ntk = (n + kKeys - 1) / kKeys;
     for (int kt = 0; kt < ntk; ++kt, ++u) {
       const int ab = 2 * eg + (u & 1);
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->acc_full[ab], (u >> 1) & 1, kWaitLimit, abort,
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->acc_full[ab], (u >> 1) & 1, a.wait_limit, abort,
                                                    a.status, 0x238));
       if (!ok) continue;
       tc_fence_after();
@@ -326,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tl.bad || tl.npow2 > a.npow2_max) continue;
         for (int v = 0; v < R && ok; ++v, ++qc) {
           const int slot = qc % QS, use = qc / QS;
-          if (use >= 1) ok = mbar_wait(&bars->q_empty[slot], (use - 1) & 1, kWaitLimit, abort, a.status, 0x230);
+          if (use >= 1) ok = mbar_wait(&bars->q_empty[slot], (use - 1) & 1, a.wait_limit, abort, a.status, 0x230);
           if (!ok) break;
           mbar_arrive_expect_tx(&bars->q_full[slot], S::QSLOT);
           // rows outside the tile's present rows (or the tensor) are loaded but never summed
@@ -350,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row0 = tl.kv * a.nkb_total + tl.kb0;
         for (int kt = 0; kt < ntk && ok; ++kt, ++kc) {
           const int slot = kc % kKStages, use = kc / kKStages;
-          if (use >= 1) ok = mbar_wait(&bars->k_empty[slot], (use - 1) & 1, kWaitLimit, abort, a.status, 0x231);
+          if (use >= 1) ok = mbar_wait(&bars->k_empty[slot], (use - 1) & 1, a.wait_limit, abort, a.status, 0x231);
           if (!ok) break;
           mbar_arrive_expect_tx(&bars->k_full[slot], S::KSLOT);
           // key blocks past the row's candidates are loaded but never read
@@ -372,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tl.bad || tl.npow2 > a.npow2_max) continue;
       const int buf = tcount & 1;
       if (tcount >= 2)
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->a_empty[buf], ((tcount >> 1) - 1) & 1, kWaitLimit,
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->a_empty[buf], ((tcount >> 1) - 1) & 1, a.wait_limit,
                                                      abort, a.status, 0x232));
       unsigned char* amat = sA + buf * S::ASLOT;
       // the sub-row sums of head mt go through shared memory (double-buffered across tiles)
@@ -380,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int v = half; v < R; v += 2) {
         const int c = qc + v, slot = c % QS;
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->q_full[slot], (c / QS) & 1, kWaitLimit, abort,
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&bars->q_full[slot], (c / QS) & 1, a.wait_limit, abort,
                                                      a.status, 0x233));
         if (ok && active) {
           // sub-row v: rows 16v .. 16v + 15 of the tile, summed token by token (present rows
@@ -442,16 +441,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile tl = cached_tile<GT>(a, tiles, tile);
         if (tl.bad || tl.npow2 > a.npow2_max) continue;
         const int buf = tcount & 1, eg = tcount & 1;   // the tile's B-operand buffer and epilogue group
-        ok = mbar_wait(&bars->a_full[buf], (tcount >> 1) & 1, kWaitLimit, abort, a.status, 0x234);
+        ok = mbar_wait(&bars->a_full[buf], (tcount >> 1) & 1, a.wait_limit, abort, a.status, 0x234);
         if (!ok) break;
         const uint32_t a_base = smem_u32(sA + buf * S::ASLOT);
         const int ntk = (tl.n + kKeys - 1) / kKeys;
         for (int kt = 0; kt < ntk; ++kt, ++kc) {
           const int slot = kc % kKStages;
           const int u = accg[eg], ab = 2 * eg + (u & 1);
-          ok = mbar_wait(&bars->k_full[slot], (kc / kKStages) & 1, kWaitLimit, abort, a.status, 0x235);
+          ok = mbar_wait(&bars->k_full[slot], (kc / kKStages) & 1, a.wait_limit, abort, a.status, 0x235);
           if (ok && u >= 2)
-            ok = mbar_wait(&bars->acc_empty[ab], ((u >> 1) - 1) & 1, kWaitLimit, abort, a.status, 0x236);
+            ok = mbar_wait(&bars->acc_empty[ab], ((u >> 1) - 1) & 1, a.wait_limit, abort, a.status, 0x236);
           if (!ok) break;
           tc_fence_after();
           const uint32_t k_base = smem_u32(sK + slot * S::KSLOT);

@@ -2,8 +2,9 @@
 
 * Argument errors are caught on the host before anything is enqueued.
 * A pipeline wait cap far too small for the pipeline makes the attention
-  kernel record COSA_ERR_TIMEOUT, drain its own copies and MMAs, free TMEM
-  and return; the context stays usable and the next call is correct.
+  kernel, and the persistent proxy kernel, record COSA_ERR_TIMEOUT, drain
+  their own copies and MMAs, free TMEM and return; the context stays usable
+  and the next call is correct.
 * A block index outside the sequence is caught by the kernels' bounds checks
   (reported as COSA_ERR_DEVICE; the access is skipped).
 """
@@ -65,6 +66,27 @@ def test_injected_wait_timeout_is_reported_and_recoverable():
     ref = osk.osk(w.q, w.k_pages, w.v_pages, w.page_table, w.seqlens, 2, 128, ref_sel["order"],
                   ref_sel["count"], 1e-4)
     gu.compare_attn(res, ref, w, 1e-4, gu.all_units(w))
+
+
+def test_injected_wait_timeout_in_the_proxy_is_reported_and_recoverable():
+    """The same for the persistent proxy kernel (head_dim 128, budget cut): every role's
+    wait gives up, the CTA drains its copies and MMAs and frees TMEM, the selection kernels
+    run on whatever was written (in bounds), the status reports the timeout, and the next
+    call is bit-exact."""
+    w, d = _case()
+    ws, kmax = cosa.alloc_workspace(d["batch"], 0.25)
+    try:
+        cosa.set_wait_limit(1)
+        cosa.proxy(d["batch"], d["q"], d["k_pages"], d["page_table"], 0.25, kmax, ws)
+        with pytest.raises(cosa.CosaError) as e:
+            cosa.check(ws)
+        assert e.value.code == 5
+    finally:
+        cosa.set_wait_limit(0)
+    got, kmax2, _ = gu.run_proxy(d, 0.25)
+    ref = kap.kap_proxy(w.q, w.k_pages, w.page_table, w.seqlens, 2, 128, 0.25)
+    assert kmax2 == ref["kmax"]
+    gu.assert_proxy_equal(got, ref)
 
 
 def test_out_of_range_block_is_caught_by_bounds_checks():
