@@ -169,13 +169,18 @@ COSA_API int cosa_workspace_init(void* workspace, size_t ws_bytes, cosa_stream_t
  *   q-block sum    = the sub-row sums folded in order from +0;
  *   int8 quantisation per vector: M = max|v|, zero if M < 2^-126, else
  *     q = rint(v * (127 / M)) (round half to even);
- *   dot = exact integer dot product; score = fp32(dot) * (M_k / 127) / n_tok;
+ *   dot = exact integer dot product; score = fp32(dot) * ks with the key
+ *     block's scale ks = (M_k / 127) / n_tok, each step one fp32 operation;
  *   HRM: key block j is HRM iff it is the argmax over j' <= i (lowest index
  *     on ties) of some valid sub-row's score;
  *   order: (HRM first, score descending, block index ascending), first k_i.
- * The workspace holds the pooled int8 keys and query vectors between the
- * three kernels the call enqueues (key pooling, query pooling, scoring and
- * selection).
+ * The workspace carries the pooled int8 keys and the intermediate results
+ * between the kernels the call enqueues.  At head_dim 128: key pooling; one
+ * persistent kernel that pools the queries, scores and finds the HRM blocks
+ * (each row's candidate score bits and HRM blocks to the workspace); the
+ * selection in registers, then the rows it leaves.  Otherwise: key pooling,
+ * query pooling (the int8 query vectors to the workspace), then scoring and
+ * selection in one kernel.  Both give identical lists.
  */
 COSA_API int cosa_proxy(const cosa_shape_t* shape, const void* q, const void* k_pages,
                const int32_t* page_table, float budget, int32_t kmax,
