@@ -90,6 +90,17 @@ __device__ __forceinline__ Tile tile_at(const ScoreArgs& a, int tile) {
   return t;
 }
 
+// Two fp32 round-to-nearest products in one packed instruction (each exactly __fmul_rn).
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 // x with bits [pos, pos + 8) replaced by the low 8 bits of v.
 __device__ __forceinline__ uint32_t bfi8(uint32_t v, uint32_t x, int pos) {
   uint32_t d;

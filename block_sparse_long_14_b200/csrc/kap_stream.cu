@@ -187,12 +187,22 @@ __device__ __forceinline__ void stream_epilogue(const ScoreArgs& a, const Stream
           if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);   // the accumulator may be overwritten
         }
         if (j < n) {
+          // the scores of the 16 columns, two round-to-nearest products per packed instruction
+          float svs[16];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const float2 p = mul_f32x2(make_float2(static_cast<float>(static_cast<int>(r[e])),
+                                                   static_cast<float>(static_cast<int>(r[e + 1]))),
+                                       make_float2(ksj, ksj));
+            svs[e] = p.x;
+            svs[e + 1] = p.y;
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int col = c * 16 + e;
             if (col >= S::NV) continue;
             const int mt = col / (R + 1), v = col % (R + 1);
-            const float sv = __fmul_rn(static_cast<float>(static_cast<int>(r[e])), ksj);
+            const float sv = svs[e];
             if (v == 0) {
               cand_row[mt * cand_head + j] = score_bits(sv);
             } else {
@@ -389,16 +399,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int rr = 0; rr < 16; ++rr) raw[rr] = *reinterpret_cast<const uint2*>(src + rr * (GT * kD * 2));
           const int lo_row = tl.rlo - 16 * v, hi_row = tl.rhi - 16 * v;   // present rows [lo_row, hi_row)
-          float sub[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          // two fp32 round-to-nearest adds per packed instruction, each dimension in token order
+          float2 s01 = make_float2(0.0f, 0.0f), s23 = make_float2(0.0f, 0.0f);
+          if (lo_row <= 0 && hi_row >= 16) {   // the whole sub-row is present
 #pragma unroll
-          for (int rr = 0; rr < 16; ++rr) {
-            if (rr >= lo_row && rr < hi_row) {
-              sub[0] = __fadd_rn(sub[0], __uint_as_float(raw[rr].x << 16));
-              sub[1] = __fadd_rn(sub[1], __uint_as_float(raw[rr].x & 0xFFFF0000u));
-              sub[2] = __fadd_rn(sub[2], __uint_as_float(raw[rr].y << 16));
-              sub[3] = __fadd_rn(sub[3], __uint_as_float(raw[rr].y & 0xFFFF0000u));
+            for (int rr = 0; rr < 16; ++rr) {
+              s01 = add_f32x2(s01, make_float2(__uint_as_float(raw[rr].x << 16), __uint_as_float(raw[rr].x & 0xFFFF0000u)));
+              s23 = add_f32x2(s23, make_float2(__uint_as_float(raw[rr].y << 16), __uint_as_float(raw[rr].y & 0xFFFF0000u)));
+            }
+          } else {
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+              if (rr >= lo_row && rr < hi_row) {
+                s01 = add_f32x2(s01, make_float2(__uint_as_float(raw[rr].x << 16), __uint_as_float(raw[rr].x & 0xFFFF0000u)));
+                s23 = add_f32x2(s23, make_float2(__uint_as_float(raw[rr].y << 16), __uint_as_float(raw[rr].y & 0xFFFF0000u)));
+              }
             }
           }
+          float sub[4] = {s01.x, s01.y, s23.x, s23.y};
           *reinterpret_cast<float4*>(sums + v * kD) = make_float4(sub[0], sub[1], sub[2], sub[3]);
           float M;
           const uint32_t packed = quantize4(sub, M);
