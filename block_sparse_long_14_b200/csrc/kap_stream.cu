@@ -101,7 +101,7 @@ __device__ __forceinline__ uint32_t quantize4(const float (&x)[4], float& M_out)
   uint32_t packed = 0;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const int q = static_cast<int>(rintf(__fmul_rn(x[e], inv)));
+    const int q = __float2int_rn(__fmul_rn(x[e], inv));   // to nearest, ties to even (= rint)
     packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * e);
   }
   M_out = M;
@@ -430,15 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // even warp once the odd one has written its sums
       named_bar_sync(kHeadBar0 + mt, 64);
       if (ok && active && half == 0) {
-        float blk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float2 b01 = make_float2(0.0f, 0.0f), b23 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int v = 0; v < R; ++v) {
           const float4 t = *reinterpret_cast<const float4*>(sums + v * kD);
-          blk[0] = __fadd_rn(blk[0], t.x);
-          blk[1] = __fadd_rn(blk[1], t.y);
-          blk[2] = __fadd_rn(blk[2], t.z);
-          blk[3] = __fadd_rn(blk[3], t.w);
+          b01 = add_f32x2(b01, make_float2(t.x, t.y));
+          b23 = add_f32x2(b23, make_float2(t.z, t.w));
         }
+        float blk[4] = {b01.x, b01.y, b23.x, b23.y};
         float M;
         const uint32_t packed = quantize4(blk, M);
         store_vec(amat, mt * (R + 1), lane, packed);
