@@ -6,31 +6,34 @@
 // group first, then the rest, each by score, cut to the stage-1 budget).
 //
 // One CTA per SM walks its share of the tiles (q-block x group of GT query
-// heads sharing a kv head, longest rows first).  The work of a tile moves
-// through warp roles connected by mbarriers, so that consecutive tiles
-// overlap: while the epilogue warps rank and select tile X, the pooling
-// warps already sum the query rows of tile X+1, whose chunks stream in by TMA.
+// heads sharing a kv head, longest rows first), described once into shared
+// memory.  The work of a tile moves through warp roles connected by
+// mbarriers, so that consecutive tiles overlap: while an epilogue group ranks
+// tile X, the pooling warps already sum the query rows of tile X+1, whose
+// chunks stream in by TMA.
 //   warp 0      Q producer: the tile's rows in chunks of 16 (one sub-row,
-//               GT heads x 128 dims, 4 KiB per head) into a ring of QS slots.
+//               GT heads x 128 dims, 4 KiB per head) into an even ring of QS
+//               slots (chunk c: slot c % QS, pooling warps of parity c % 2).
 //   warp 1      key producer: the pooled int8 key blocks of the tile's kv head,
 //               128 blocks (16 KiB, 128B swizzle) per score tile, 3 slots.
-//   warps 2-5   pooling, one query head each: the fp32 sum of each 16-row
-//               sub-row token by token, the q-block sum as their fold, int8
-//               quantisation, written as the MMA's B operand (double-buffered
-//               across tiles).
-//   warp 6      MMA issuer: D[j][v] = Kq_j . q_v (s8 x s8 -> exact s32) with
+//   warps 2-9   pooling, two warps per query head taking the even and the odd
+//               sub-rows: the fp32 sum of each 16-row sub-row token by token,
+//               its int8 quantisation written as the MMA's B operand
+//               (double-buffered across tiles); the even warp then folds the
+//               head's sub-row sums in order into the q-block vector.
+//   warp 10     MMA issuer: D[j][v] = Kq_j . q_v (s8 x s8 -> exact s32) with
 //               tcgen05 kind::i8, 128 key blocks in M (one TMEM lane each) and
-//               the tile's GT (R + 1) vectors in N, into one of two TMEM
-//               accumulators.
-//   warps 7-14  epilogue, two groups of four warps (TMEM lane quadrants 3, 0,
+//               the tile's GT (R + 1) vectors in N, into one of the two TMEM
+//               accumulators of the tile's epilogue group.
+//   warps 11-18 epilogue, two groups of four warps (TMEM lane quadrants 3, 0,
 //               1, 2 and 3, 0, 1, 2) taking alternate tiles: each lane turns
 //               one key block's dots into its score bits per head (written to
-//               the workspace row of that head) and updates the sub-rows'
+//               the workspace row of that head) and keeps the sub-rows'
 //               running argmax; the group then reduces the argmax to the HRM
 //               blocks of each head (written next to the scores).
-// The selection runs in its own kernel (select_rows_kernel): one warp per
-// (head, q-block) row, many rows per SM, a sampled threshold and a sort of the
-// few keys below it (a radix select when that does not fit).
+// The selection runs in its own kernels: select_fast_kernel, one warp per
+// (head, q-block) row, many rows per SM, a sampled threshold and a register
+// sort of the few keys below it; select_rows_kernel for the rows it leaves.
 // Scores, flags and lists are bit-identical to the two-stage kernels: the same
 // fp32 operations in the same order, and integer dots.  Every wait is bounded;
 // on expiry the CTA records COSA_ERR_TIMEOUT, lets its own copies and MMAs
